@@ -1,0 +1,180 @@
+/*
+ * segpaged.h -- C ABI of the SegPagedAttention library for NVIDIA B200 (sm_100a).
+ *
+ * SegPagedAttention stores the KV cache as pages keyed by (layer, head, segment) instead of a
+ * dense [B, H, L, D] tensor. A global head keeps its whole context; a local head physically keeps
+ * only its sink tokens and its recent window. One mask-free, variable-length attention kernel runs
+ * every head over exactly its own ragged KV.
+ *   Sources: "小红书把 KV Cache 按「头」拆了" (zhichai.net), 事件内容 item 3 "SegPagedAttention 存储";
+ *   "RedKnot – 小红书研发并开源的长上下文大模型推理引擎" (shshi.cn), 技术原理 1 "SegPagedAttention存储架构";
+ *   "为什么长上下文推理这么慢？RedKnot…" (bjdmk.com.cn), 二 "三大核心机制" item 3;
+ *   "RedKnot - Xiaohongshuが開発した…" (aiboss88.com), 技術原則, item on paged storage removing the
+ *   attn_mask kernel penalty.
+ *
+ * The calls follow the four adapters the last page names (使い方): BUILDSTATE -> segpaged_build,
+ * SELECTVISIBLESTATE -> segpaged_prefill_plan, EXECUTE -> segpaged_attn_prefill; PROFILE (the
+ * offline head classification) happens outside this library and reaches it as the class map.
+ *
+ * Conventions shared by every call
+ *  - Visibility. Query position i of a sequence sees key j iff j <= i and (the KV head is global, or
+ *    j < sink, or j > i - window). Queries are the Lq tail positions L-Lq .. L-1 of a sequence of
+ *    context length L. Query head h reads KV head h / G, G = num_q_heads / num_kv_heads.
+ *  - Stored pages. Logical page n of a (sequence, KV head) holds tokens [n*P, n*P+P). A global head
+ *    stores pages 0 .. ceil(L/P)-1. A local head stores the pages holding a token < min(sink, L) and
+ *    the pages holding a token >= max(L - Lq - window + 1, 0). The page table of a (sequence, KV
+ *    head) lists the physical page of each stored logical page in ascending logical order
+ *    (sink pages first, then window pages). Physical ids may be any permutation.
+ *  - Layouts (row-major, bf16 unless stated): dense K/V [sum L_b, Hkv, D]; Q and O
+ *    [sum Lq_b, Hq, D]; LSE float32 [Hq, sum Lq_b] (natural log); pools [num_pages, P, D].
+ *  - Page-table arrays are flattened over (sequence b, KV head k) in b-major order: entries of head
+ *    (b, k) are page_table[offs[b*Hkv + k] .. offs[b*Hkv + k + 1]).
+ *  - Ownership. Every pointer is owned by the caller; the library keeps none after a call returns
+ *    and allocates no device memory. "dev" pointers are device memory, "host" pointers host memory.
+ *  - Streams. Device work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream) and is asynchronous to the host.
+ *  - Errors. A call returns 0 (or a count) on success and a negative SEGPAGED_ERR_* code otherwise;
+ *    on a host-detected error nothing is enqueued. Device-side checks (a page id outside
+ *    [0, num_pages), a page table whose length disagrees with the storage rule, a pipeline wait that
+ *    timed out) OR a SEGPAGED_STATUS_* bit into the optional device status word and keep all
+ *    memory accesses in bounds; the caller reads the word after synchronising.
+ *  - Supported shapes: head_dim in {64, 128}; page_size in {16, 32, 64, 128}; G a power of two
+ *    <= 128; base pointers of q, pools and o 16-byte aligned.
+ */
+#ifndef SEGPAGED_H
+#define SEGPAGED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SEGPAGED_OK 0
+#define SEGPAGED_ERR_NULL (-1)      /* a required pointer is NULL */
+#define SEGPAGED_ERR_DIMS (-2)      /* unsupported or inconsistent dims */
+#define SEGPAGED_ERR_CLASS (-3)     /* head class out of range (sink < 0, window < 1 for a local head) */
+#define SEGPAGED_ERR_SEQ (-4)       /* negative length, or Lq > L */
+#define SEGPAGED_ERR_PAGES (-5)     /* page-table offsets disagree with the storage rule */
+#define SEGPAGED_ERR_CAPACITY (-6)  /* output array too small */
+#define SEGPAGED_ERR_CUDA (-7)      /* a CUDA runtime/driver call failed */
+#define SEGPAGED_ERR_ALIGN (-8)     /* a base pointer is not 16-byte aligned */
+
+#define SEGPAGED_STATUS_PAGE_ID 1   /* a page id was outside [0, num_pages); it was clamped */
+#define SEGPAGED_STATUS_TABLE 2     /* a head's page-table length disagreed with the storage rule */
+#define SEGPAGED_STATUS_TIMEOUT 4   /* a pipeline wait gave up; outputs of this call are undefined */
+#define SEGPAGED_STATUS_UNIT 8      /* a work unit referenced entries past the page table */
+
+typedef struct {
+  int32_t num_seqs;      /* B */
+  int32_t num_q_heads;   /* Hq */
+  int32_t num_kv_heads;  /* Hkv; Hq % Hkv == 0 */
+  int32_t head_dim;      /* D */
+  int32_t page_size;     /* P, tokens per page */
+  int32_t num_pages;     /* physical pages in each of k_pool and v_pool */
+} segpaged_dims;
+
+/* Class of one (sequence, KV head) of one layer: the offline head classification. */
+typedef struct {
+  int32_t is_global;  /* 1: full causal context; 0: local */
+  int32_t sink;       /* S >= 0, local heads only */
+  int32_t window;     /* W >= 1, local heads only */
+} segpaged_head_class;
+
+/* One prefill work unit: a (sequence, KV head, query tile) with its visible page ranges.
+ * Produced by segpaged_prefill_plan; its fields are private to the library. 64 bytes. */
+typedef struct {
+  int32_t v[16];
+} segpaged_unit;
+
+/* Text for an error code (static storage). */
+const char* segpaged_error_string(int code);
+
+/*
+ * Physical KV footprint of a layer (host only, no device work).
+ *   ctx_len[B], q_len[B] (host): L_b and Lq_b.  cls[B*Hkv] (host).
+ *   pages_per_head[B*Hkv] (host, nullable): stored page count of each (b, k).
+ *   dense_bytes (host, nullable): K+V bytes if every KV head kept all ceil(L_b/P) pages.
+ * Returns the stored K+V bytes (num stored pages * P * D * 2 tensors * 2 bytes), or an error code.
+ * Source: the physically sparse access of SegPagedAttention, which cuts the KV bytes moved
+ * (shshi.cn, 技术原理 1, "物理级稀疏访问").
+ */
+int64_t segpaged_pages_bytes(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                             const segpaged_head_class* cls, int64_t* dense_bytes, int32_t* pages_per_head);
+
+/*
+ * RoPE re-alignment table (host only). out[b][d][0..1] = (cos, sin) of deltas[b] * theta^(-2d/D),
+ * d in [0, D/2), evaluated in double and rounded to float. out is host [num_seqs, D/2, 2].
+ * Source: rotating offline-computed keys from their original to their actual position
+ * (shshi.cn, 技术原理 2 "位置无关缓存复用", item "RoPE位置对齐").
+ */
+int segpaged_rope_cos_sin(double theta, const int32_t* deltas, int32_t num_seqs, int32_t head_dim, float* out);
+
+/*
+ * BUILDSTATE: scatter a layer's dense K/V into the page pools (one kernel launch).
+ *   k_dense, v_dense (dev): [sum L_b, Hkv, D] bf16.   cu_seqlens_k (dev) [B+1]: token offsets.
+ *   q_len (dev) [B]: Lq_b, which fixes the window pages a local head stores.  cls (dev) [B*Hkv].
+ *   page_table (dev, int32) and page_table_offs (dev, int32 [B*Hkv+1]) as described above.
+ *   rope_cos_sin (dev, nullable) [B, D/2, 2] float from segpaged_rope_cos_sin: when set, every
+ *     stored key is rotated (rotate-half pairs (d, d+D/2)): y1 = x1*c - x2*s, y2 = x2*c + x1*s,
+ *     each product and sum rounded to float, then rounded to bf16 (nearest even). V is copied as is.
+ *   k_pool, v_pool (dev) [num_pages, P, D] bf16: each stored page receives its P rows; rows past
+ *     L_b are written as zero. Pages not named by any table are not touched.
+ *   status (dev, nullable): see SEGPAGED_STATUS_*.
+ * Sources: the BUILDSTATE adapter, which precomputes fragment KV and stores it page by page per head
+ *   into the global/local pools (aiboss88.com, 使い方, second item); the RoPE re-alignment
+ *   (shshi.cn, 技术原理 2, item "RoPE位置对齐").
+ */
+int segpaged_build(const segpaged_dims* dims, const void* k_dense, const void* v_dense,
+                   const int32_t* cu_seqlens_k, const int32_t* q_len, const segpaged_head_class* cls,
+                   const int32_t* page_table, const int32_t* page_table_offs, const float* rope_cos_sin,
+                   void* k_pool, void* v_pool, int32_t* status, void* stream);
+
+/*
+ * SELECTVISIBLESTATE: plan the prefill work (host only).
+ * Splits every (sequence, KV head) into query tiles of 128/G positions x G query heads, records for
+ * each tile the page ranges its queries can see (the sink pages and the window pages, in page-table
+ * index space) and sorts the units by their number of 128-key tiles, longest first.
+ *   ctx_len, q_len (host) [B]; cls (host) [B*Hkv]; page_table_offs (host) [B*Hkv+1] (the same
+ *   offsets later given to the device), checked against the storage rule.
+ *   units (host, nullable) [capacity].
+ * Returns the number of units (also when units is NULL, to size the array), or an error code.
+ * The caller copies the units to device memory for segpaged_attn_prefill; a plan stays valid for
+ * any call with the same lengths, classes and offsets (e.g. every layer sharing a class map).
+ * Source: the SELECTVISIBLESTATE adapter, which picks the local-head KV to reuse and the global-head
+ *   ranges to compute (aiboss88.com, 使い方, third item).
+ */
+int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                              const segpaged_head_class* cls, const int32_t* page_table_offs,
+                              segpaged_unit* units, int64_t capacity);
+
+/* Device scratch bytes segpaged_attn_prefill needs (the work-unit counter). */
+size_t segpaged_prefill_workspace_bytes(int64_t num_units);
+
+/*
+ * EXECUTE: causal attention of every query head over its own ragged paged KV (one persistent
+ * kernel launch, preceded by a 4-byte memset of the workspace).
+ *   q (dev) [total_q, Hq, D] bf16.  k_pool, v_pool (dev) [num_pages, P, D] bf16.
+ *   page_table (dev, int32) [page_table_len].  units (dev) [num_units] from segpaged_prefill_plan.
+ *   softmax_scale: logits are scale * q.k (1/sqrt(D) in the usual case).
+ *   o (dev) [total_q, Hq, D] bf16: O = softmax(logits over the visible keys) . V.
+ *   lse (dev) [Hq, total_q] float: natural-log sum of exp(logits) over the visible keys.
+ *   workspace (dev) >= segpaged_prefill_workspace_bytes(num_units), 16-byte aligned.
+ *   status (dev, nullable): see SEGPAGED_STATUS_*.
+ * Every stored page slot must hold finite values (segpaged_build writes zeros past the context end).
+ * Sources: one fused variable-length attention kernel that keeps every head on the fast path and
+ *   builds no attention mask (zhichai.net, 事件内容 item 3); global heads read all context pages and
+ *   local heads only their sink and recent-window pages, run by a mask-free varlen kernel
+ *   (bjdmk.com.cn, 二 item 3); the EXECUTE adapter (aiboss88.com, 使い方, fourth item).
+ */
+int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q,
+                          const void* k_pool, const void* v_pool, const int32_t* page_table,
+                          int64_t page_table_len, const segpaged_unit* units, int64_t num_units,
+                          float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                          int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEGPAGED_H */
