@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the SegPagedAttention hot path on B200.
+
+A step is one pass of the whole hot path over every layer of the workload: storage accounting and
+work planning on the host, the build scatter of the layer's K/V into its pages, and the mask-free
+paged prefill. The metric is visible-KV TFLOP/s: 4 * D * sum |V(i)| over every (query row, query head)
+of every layer, divided by the step time (CUDA events, max over ranks).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun every rank runs its own replica of the workload (rank-specific seeds, no data-path
+collective: weak scaling); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "visible-KV TFLOP/s and ms per layer for SegPagedAttention prefill; % roofline"
+DEFAULT_WORKLOAD = "dsv4-flash"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["head_sparse_paged_b200/csrc/prefill_sm100.cuh", "head_sparse_paged_b200/csrc/sm100_ptx.cuh",
+                  "head_sparse_paged_b200/csrc/plan.h"]
+
+
+# ----------------------------------------------------------------------------------- utilities
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle sample")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (host-side reporting only; not on the data path)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(name: str, rank: int):
+    """The workload of one rank: same shapes, rank-specific seed (independent replicas)."""
+    from head_sparse_paged_b200 import synth
+    w = synth.get(name)
+    if rank:
+        w = dataclasses.replace(w, seed=w.seed + 100003 * rank)
+    return w
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch(workload: str):
+    """DRAM bytes per prefill launch from the committed ncu summary, if it was taken on the current
+    kernel sources for this workload; else None."""
+    p = os.path.join(ROOT, "profiles", f"prefill_traffic_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_sources_sha256") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every 100 ms while active."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:   # the NVML handle of the physical GPU behind this CUDA device
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self._reasons_fn(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------ oracle timing
+
+def oracle_sample(w, inputs_for_head, seconds: float, seed: int = 0):
+    """Times the fp64 oracle on a bounded, seeded sample of the workload's (row, query head) items.
+
+    inputs_for_head(layer, b, kh) -> oracle Problem of that (sequence, KV head). Items are drawn from
+    every layer class present, in rounds, until the time budget is spent. Returns (visible TFLOP/s,
+    sample description, threads)."""
+    import numpy as np
+    from head_sparse_paged_b200.runner import visible_counts
+    from oracle import reference as orc
+
+    lib = orc.OracleLib()
+    rng = np.random.default_rng(seed)
+    kinds = {}
+    for li in range(w.layers):                       # one layer of each kind (number of global heads)
+        kinds.setdefault(int(w.classes[li][..., 0].sum()), li)
+    layers = sorted(kinds.values())
+    done_flops, spent, items_done = 0.0, 0.0, 0
+    scale = 1.0 / math.sqrt(w.head_dim)
+    cache = {}
+    t_end = time.time() + seconds
+    rounds = 0
+    while time.time() < t_end and rounds < 64:
+        rounds += 1
+        for li in layers:
+            b = int(rng.integers(w.num_seqs))
+            kh = int(rng.integers(w.num_kv_heads))
+            key = (li, b, kh)
+            if key not in cache:
+                if len(cache) > 8:
+                    cache.pop(next(iter(cache)))
+                cache[key] = inputs_for_head(li, b, kh)
+            pb = cache[key]
+            Lq = w.q_lens[b]
+            rows = rng.integers(0, Lq, size=8)
+            items = np.array([(int(r), h) for r in rows for h in range(w.group)], np.int64)
+            cnt = visible_counts(w, li, b, kh)
+            t0 = time.perf_counter()
+            lib.attention(pb, scale, items)
+            spent += time.perf_counter() - t0
+            done_flops += 4.0 * w.head_dim * float(sum(cnt[int(r)] for r in rows)) * w.group
+            items_done += len(items)
+            if time.time() >= t_end:
+                break
+    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    desc = (f"{items_done} (query row, head) items of layers {layers} drawn at random, timed {spent:.1f} s; "
+            f"fp64 C oracle, OpenMP over items")
+    return done_flops / spent / 1e12, desc, threads
+
+
+def oracle_head_inputs_from_synth(w):
+    """Oracle inputs regenerated on the CPU from the seeded generators (used by --impl reference)."""
+    import numpy as np
+    import torch
+    from head_sparse_paged_b200 import synth
+    from oracle import reference as orc
+
+    dense = {}
+
+    def get(li, b, kh):
+        src = 0 if w.layers > 1 else li
+        if src not in dense:
+            q, k, v = synth.layer_inputs(w, src, device="cpu")
+            dense[src] = (k, v)
+        k, v = dense[src]
+        q = synth.layer_inputs(w, li, device="cpu", parts="q")[0]
+        return _head_problem(w, li, b, kh, q, k, v)
+
+    return get
+
+
+def _head_problem(w, li, b, kh, q, k, v):
+    import numpy as np
+    from oracle import reference as orc
+    G = w.group
+    cq, ck = w.cu_q(), w.cu_k()
+    qs = q[cq[b]:cq[b + 1], kh * G:(kh + 1) * G].float().cpu().numpy()
+    ks = k[ck[b]:ck[b + 1], kh:kh + 1].float().cpu().numpy()
+    vs = v[ck[b]:ck[b + 1], kh:kh + 1].float().cpu().numpy()
+    if w.rope_theta is not None:
+        ks = orc.rope_rotate_bf16(ks, orc.rope_cos_sin(w.rope_theta, [w.rope_deltas[b]], w.head_dim)[0])
+    g, S, W = (int(x) for x in w.classes[li, b, kh])
+    return orc.Problem(qs, ks, vs, np.array([0, w.q_lens[b]], np.int32), np.array([0, w.ctx_lens[b]], np.int32),
+                       np.array([[g]]), np.array([[S]]), np.array([[W]]))
+
+
+# -------------------------------------------------------------------------------------- arms
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores, on this workload's config and metric."""
+    if rank != 0:
+        return 0
+    from head_sparse_paged_b200.runner import visible_flops
+    w = rank_workload(args.workload, 0)
+    get = oracle_head_inputs_from_synth(w)
+    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, get, per_step / 4, seed=1)
+    vals = []
+    desc = threads = None
+    for s in range(args.steps):
+        v, desc, threads = oracle_sample(w, get, per_step, seed=100 + s)
+        vals.append(v)
+    value = statistics.median(vals)
+    flops = visible_flops(w)
+    ms = flops / (value * 1e12) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: {desc}; step time extrapolated by visible FLOPs"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "description": w.description, "layers": w.layers, "seq_lens": list(w.ctx_lens),
+            "q_lens": list(w.q_lens), "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "page_size": w.page_size, "page_order": w.page_order}
+
+
+def run_ours(args, rank, world, local):
+    import numpy as np
+    import torch
+    from head_sparse_paged_b200.runner import Runner, visible_flops
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = rank_workload(args.workload, rank)
+    runner = Runner(w, device=device, keep_dense=True, shared_dense=(w.layers > 1))
+    torch.cuda.synchronize()
+    runner.check_status()
+    flops_layer = {li: visible_flops(w, [li]) for li in runner.layers}
+    flops_step = sum(flops_layer.values())
+    stream = torch.cuda.current_stream()
+    n_layers = len(runner.layers)
+
+    # per-prefill-launch events (on the launching stream) for the dominant kernel's roofline
+    ev = {}
+
+    def mark(li, start):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        ev.setdefault(li, []).append(e)
+
+    for _ in range(args.warmup):
+        runner.full_step()
+    torch.cuda.synchronize()
+    runner.check_status()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            runner.full_step(on_prefill=mark)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = reduce_max(t0.elapsed_time(t1), world, device)
+    runner.check_status()
+    prefill_ms = {li: [ev[li][2 * s].elapsed_time(ev[li][2 * s + 1]) for s in range(args.steps)] for li in ev}
+    prefill_total_ms = sum(sum(v) for v in prefill_ms.values())
+    ms_step = ms_total / args.steps
+    value = world * flops_step * args.steps / (ms_total * 1e-3) / 1e12
+    achieved = sum(flops_layer[li] * len(prefill_ms[li]) for li in prefill_ms) / (prefill_total_ms * 1e-3) / 1e12
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    traffic = traffic_per_launch(w.name)
+    kinds = {}
+    for li in runner.layers:
+        kinds.setdefault("all-global" if runner.state[li].cls[..., 0].all() else "mixed", []).append(li)
+    per_kind = {k: {"layers": len(v), "prefill_ms": statistics.mean(statistics.mean(prefill_ms[li]) for li in v),
+                    "visible_tflop": flops_layer[v[0]] / 1e12} for k, v in kinds.items()}
+    stored = sum(runner.state[li].stored_bytes for li in runner.layers)
+    dense = sum(runner.state[li].dense_bytes for li in runner.layers)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(runner, args, world, device, flops_step)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        def inputs(li, b, kh):
+            k, v = runner.dense_of(li)
+            return _head_problem(w, li, b, kh, runner.state[li].q, k, v)
+        v_cpu, desc, threads = oracle_sample(w, inputs, args.cpu_seconds)
+        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank != 0:
+        return 0
+    cfg = workload_config(w)
+    cfg.update({"global_batch": w.num_seqs * world, "parallelism": f"replicas x{world}" if world > 1 else "single",
+                "l2": f"inputs larger than L2 (page pool {runner.num_pages * w.page_size * w.head_dim * 4 / 1e9:.1f} GB, "
+                      f"stored per step {stored / 1e9:.2f} GB)",
+                "dense_kv_source": "shared by all layers" if runner.shared_dense else "per layer"})
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "ms_per_layer": prefill_total_ms / args.steps / n_layers,
+        "prefill_ms_by_layer_kind": per_kind,
+        "kv_bytes": {"segpaged": stored, "dense": dense, "ratio": dense / max(stored, 1)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{src} bf16_tflops_sustained", "kernel": "segpaged_prefill_kernel"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * n_layers * 2,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def measure_e2e(runner, args, world, device, flops_step):
+    """Same metric through the public API with host buffers: every step copies the queries of every
+    layer and the work plan from pinned host memory and reads O and LSE back into pinned host memory."""
+    import torch
+    q_host = {li: runner.state[li].q.cpu().pin_memory() for li in runner.layers}
+    o_host = {li: torch.empty_like(runner.state[li].o, device="cpu").pin_memory() for li in runner.layers}
+    l_host = {li: torch.empty_like(runner.state[li].lse, device="cpu").pin_memory() for li in runner.layers}
+    h2d = sum(q_host[li].numel() * 2 + runner.state[li].units.nbytes for li in runner.layers)
+    d2h = sum(o_host[li].numel() * 2 + l_host[li].numel() * 4 for li in runner.layers)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for li in runner.layers:
+            runner.state[li].q.copy_(q_host[li], non_blocking=True)
+        runner.full_step()
+        for li in runner.layers:
+            o_host[li].copy_(runner.state[li].o, non_blocking=True)
+            l_host[li].copy_(runner.state[li].lse, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    steps = max(1, min(args.steps, 5))
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max(t0.elapsed_time(t1), world, device)
+    return {"value": world * flops_step * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        return run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

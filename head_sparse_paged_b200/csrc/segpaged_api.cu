@@ -1,0 +1,354 @@
+// segpaged_api.cu -- host side of the SegPagedAttention C ABI (see include/segpaged.h).
+//
+// Argument validation, the storage accounting (segpaged_pages_bytes), the RoPE table, the work
+// planner (segpaged_prefill_plan, the SELECTVISIBLESTATE step), TMA tensor-map encoding and the
+// kernel launches. The library allocates no device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/segpaged.h"
+#include "build_kernel.cuh"
+#include "plan.h"
+#include "prefill_sm100.cuh"
+
+using namespace segpaged;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int device_sm_count(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map, innermost dimension first, 128-byte swizzle.
+bool encode_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1,
+               uint32_t b2) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const segpaged_dims* d) {
+  if (!d) return SEGPAGED_ERR_NULL;
+  if (d->num_seqs < 0 || d->num_kv_heads < 1 || d->num_q_heads < 1 || d->num_q_heads % d->num_kv_heads != 0)
+    return SEGPAGED_ERR_DIMS;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  if (G > 128 || (G & (G - 1)) != 0) return SEGPAGED_ERR_DIMS;
+  if (d->head_dim != 64 && d->head_dim != 128) return SEGPAGED_ERR_DIMS;
+  if (d->page_size != 16 && d->page_size != 32 && d->page_size != 64 && d->page_size != 128) return SEGPAGED_ERR_DIMS;
+  if (d->num_pages < 0) return SEGPAGED_ERR_DIMS;
+  return SEGPAGED_OK;
+}
+
+int check_class(const segpaged_head_class& c) {
+  if (c.is_global) return SEGPAGED_OK;
+  if (c.sink < 0 || c.window < 1) return SEGPAGED_ERR_CLASS;
+  return SEGPAGED_OK;
+}
+
+int log2_int(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* segpaged_error_string(int code) {
+  switch (code) {
+    case SEGPAGED_OK: return "ok";
+    case SEGPAGED_ERR_NULL: return "a required pointer is NULL";
+    case SEGPAGED_ERR_DIMS: return "unsupported or inconsistent dims";
+    case SEGPAGED_ERR_CLASS: return "head class out of range (sink < 0 or window < 1 for a local head)";
+    case SEGPAGED_ERR_SEQ: return "bad sequence lengths (negative, or Lq > L)";
+    case SEGPAGED_ERR_PAGES: return "page-table offsets disagree with the storage rule";
+    case SEGPAGED_ERR_CAPACITY: return "output array too small";
+    case SEGPAGED_ERR_CUDA: return "a CUDA runtime or driver call failed";
+    case SEGPAGED_ERR_ALIGN: return "a base pointer is not 16-byte aligned";
+    default: return "unknown error";
+  }
+}
+
+int64_t segpaged_pages_bytes(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                             const segpaged_head_class* cls, int64_t* dense_bytes, int32_t* pages_per_head) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->num_seqs > 0 && (!ctx_len || !q_len || !cls)) return SEGPAGED_ERR_NULL;
+  const int B = dims->num_seqs, H = dims->num_kv_heads, P = dims->page_size;
+  int64_t stored = 0, dense = 0;
+  for (int b = 0; b < B; ++b) {
+    if (ctx_len[b] < 0 || q_len[b] < 0 || q_len[b] > ctx_len[b]) return SEGPAGED_ERR_SEQ;
+    for (int k = 0; k < H; ++k) {
+      const segpaged_head_class& c = cls[b * H + k];
+      if ((rc = check_class(c))) return rc;
+      const Split s = storage_split(ctx_len[b], q_len[b], c.is_global, c.sink, c.window, P);
+      stored += s.total;
+      dense += ceil_div(ctx_len[b], P);
+      if (pages_per_head) pages_per_head[b * H + k] = s.total;
+    }
+  }
+  const int64_t unit = (int64_t)P * dims->head_dim * 2 /*K and V*/ * 2 /*bf16*/;
+  if (dense_bytes) *dense_bytes = dense * unit;
+  return stored * unit;
+}
+
+int segpaged_rope_cos_sin(double theta, const int32_t* deltas, int32_t num_seqs, int32_t head_dim, float* out) {
+  if (num_seqs < 0 || head_dim < 2 || (head_dim & 1) || !(theta > 0.0)) return SEGPAGED_ERR_DIMS;
+  if (num_seqs > 0 && (!deltas || !out)) return SEGPAGED_ERR_NULL;
+  const int half = head_dim / 2;
+  for (int b = 0; b < num_seqs; ++b)
+    for (int d = 0; d < half; ++d) {
+      const double inv_freq = std::pow(theta, -2.0 * d / head_dim);
+      const double ang = (double)deltas[b] * inv_freq;
+      out[((int64_t)b * half + d) * 2 + 0] = (float)std::cos(ang);
+      out[((int64_t)b * half + d) * 2 + 1] = (float)std::sin(ang);
+    }
+  return SEGPAGED_OK;
+}
+
+int segpaged_build(const segpaged_dims* dims, const void* k_dense, const void* v_dense, const int32_t* cu_seqlens_k,
+                   const int32_t* q_len, const segpaged_head_class* cls, const int32_t* page_table,
+                   const int32_t* page_table_offs, const float* rope_cos_sin, void* k_pool, void* v_pool,
+                   int32_t* status, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->num_seqs == 0) return SEGPAGED_OK;
+  if (!k_dense || !v_dense || !cu_seqlens_k || !q_len || !cls || !page_table || !page_table_offs || !k_pool || !v_pool)
+    return SEGPAGED_ERR_NULL;
+  if (!aligned16(k_dense) || !aligned16(v_dense) || !aligned16(k_pool) || !aligned16(v_pool) ||
+      (rope_cos_sin && !aligned16(rope_cos_sin)))
+    return SEGPAGED_ERR_ALIGN;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SEGPAGED_ERR_CUDA;
+  BuildParams p;
+  p.k_dense = static_cast<const __nv_bfloat16*>(k_dense);
+  p.v_dense = static_cast<const __nv_bfloat16*>(v_dense);
+  p.cu_k = cu_seqlens_k;
+  p.q_len = q_len;
+  p.cls = reinterpret_cast<const int32_t*>(cls);
+  p.table = page_table;
+  p.offs = page_table_offs;
+  p.cos_sin = rope_cos_sin;
+  p.k_pool = static_cast<__nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<__nv_bfloat16*>(v_pool);
+  p.status = status;
+  p.B = dims->num_seqs;
+  p.Hkv = dims->num_kv_heads;
+  p.P = dims->page_size;
+  p.num_pages = dims->num_pages;
+  const int grid = std::max(1, device_sm_count(dev)) * 8;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dims->head_dim == 128) {
+    if (rope_cos_sin) build_scatter_kernel<128, true><<<grid, 256, 0, st>>>(p);
+    else build_scatter_kernel<128, false><<<grid, 256, 0, st>>>(p);
+  } else {
+    if (rope_cos_sin) build_scatter_kernel<64, true><<<grid, 256, 0, st>>>(p);
+    else build_scatter_kernel<64, false><<<grid, 256, 0, st>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
+}
+
+int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                              const segpaged_head_class* cls, const int32_t* page_table_offs, segpaged_unit* units,
+                              int64_t capacity) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  const int B = dims->num_seqs, H = dims->num_kv_heads, P = dims->page_size;
+  if (B > 0 && (!ctx_len || !q_len || !cls || !page_table_offs)) return SEGPAGED_ERR_NULL;
+  const int G = dims->num_q_heads / H;
+  const int npos = 128 / G;
+  const int ppt = 128 / P;
+  std::vector<segpaged_unit> out;
+  int32_t qrow = 0;
+  if (page_table_offs && page_table_offs[0] != 0) return SEGPAGED_ERR_PAGES;
+  for (int b = 0; b < B; ++b) {
+    const int32_t L = ctx_len[b], Lq = q_len[b];
+    if (L < 0 || Lq < 0 || Lq > L) return SEGPAGED_ERR_SEQ;
+    const int32_t q0 = L - Lq;
+    for (int k = 0; k < H; ++k) {
+      const int bk = b * H + k;
+      const segpaged_head_class& c = cls[bk];
+      if ((rc = check_class(c))) return rc;
+      const Split sp = storage_split(L, Lq, c.is_global, c.sink, c.window, P);
+      if (page_table_offs[bk + 1] - page_table_offs[bk] != sp.total) return SEGPAGED_ERR_PAGES;
+      const bool merged = sp.n_sink == sp.total;
+      for (int32_t t0 = 0; t0 < Lq; t0 += npos) {
+        const int32_t r0 = q0 + t0, nv = std::min(npos, Lq - t0), r1 = r0 + nv - 1;
+        int32_t a_n = 0, b0 = 0, b_n = 0;
+        if (c.is_global) {
+          b_n = r1 / P + 1;
+        } else {
+          a_n = (int32_t)ceil_div(std::min<int64_t>(c.sink, (int64_t)r1 + 1), P);
+          const int32_t wlo = std::max<int64_t>((int64_t)r0 - c.window + 1, 0);
+          const int32_t lp_lo = wlo / P, lp_hi = r1 / P;
+          if (merged) {
+            if (lp_lo <= a_n) {  // sink and window ranges meet: one range from page 0
+              a_n = 0;
+              b0 = 0;
+              b_n = lp_hi + 1;
+            } else {
+              b0 = lp_lo;
+              b_n = lp_hi - lp_lo + 1;
+            }
+          } else {
+            b0 = sp.n_sink + (lp_lo - sp.w0);
+            b_n = lp_hi - lp_lo + 1;
+          }
+        }
+        segpaged_unit u;
+        std::memset(&u, 0, sizeof(u));
+        u.v[U_QROW] = qrow + t0;
+        u.v[U_POS0] = r0;
+        u.v[U_NPOS] = nv;
+        u.v[U_KVH] = k;
+        u.v[U_TOFF] = page_table_offs[bk];
+        u.v[U_NSINK] = sp.n_sink;
+        u.v[U_W0] = sp.w0;
+        u.v[U_GLOBAL] = c.is_global ? 1 : 0;
+        u.v[U_SINK] = c.is_global ? 0 : c.sink;
+        u.v[U_WIN] = c.is_global ? 0 : c.window;
+        u.v[U_AN] = a_n;
+        u.v[U_B0] = b0;
+        u.v[U_BN] = b_n;
+        u.v[U_NTILES] = (int32_t)ceil_div(a_n + b_n, ppt);
+        u.v[U_TOTAL] = sp.total;
+        u.v[U_SEQ] = b;
+        out.push_back(u);
+      }
+    }
+    qrow += Lq;
+  }
+  // Longest first, so the persistent grid finishes together; ties keep plan order.
+  std::stable_sort(out.begin(), out.end(),
+                   [](const segpaged_unit& a, const segpaged_unit& b) { return a.v[U_NTILES] > b.v[U_NTILES]; });
+  const int64_t n = (int64_t)out.size();
+  if (!units) return n;
+  if (capacity < n) return SEGPAGED_ERR_CAPACITY;
+  if (n) std::memcpy(units, out.data(), sizeof(segpaged_unit) * (size_t)n);
+  return n;
+}
+
+size_t segpaged_prefill_workspace_bytes(int64_t num_units) {
+  (void)num_units;
+  return 256;
+}
+
+}  // extern "C"
+
+namespace {
+
+template <int D, int P>
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
+                   int grid, cudaStream_t st) {
+  using C = PrefillCfg<D, P>;
+  static bool configured[kMaxDevices] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(segpaged_prefill_kernel<D, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return SEGPAGED_ERR_CUDA;
+    configured[dev] = true;
+  }
+  segpaged_prefill_kernel<D, P><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
+                                     const void* v_pool, const int32_t* page_table, int64_t page_table_len,
+                                     const segpaged_unit* units, int64_t num_units, float softmax_scale, void* o,
+                                     float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                                     void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (num_units < 0 || total_q < 0 || page_table_len < 0 || num_units > INT32_MAX) return SEGPAGED_ERR_DIMS;
+  if (num_units == 0) return SEGPAGED_OK;
+  if (!q || !k_pool || !v_pool || !page_table || !units || !o || !lse || !workspace) return SEGPAGED_ERR_NULL;
+  if (workspace_bytes < segpaged_prefill_workspace_bytes(num_units)) return SEGPAGED_ERR_CAPACITY;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o) || !aligned16(units) ||
+      !aligned16(workspace))
+    return SEGPAGED_ERR_ALIGN;
+  if (total_q < 1 || dims->num_pages < 1) return SEGPAGED_ERR_DIMS;
+  const int D = dims->head_dim, P = dims->page_size, Hq = dims->num_q_heads;
+  const int G = Hq / dims->num_kv_heads;
+  CUtensorMap tq, tk, tv;
+  if (!encode_3d(&tq, q, D, Hq, (uint64_t)total_q, 64, G, 128 / G) ||
+      !encode_3d(&tk, k_pool, D, P, (uint64_t)dims->num_pages, 64, P, 1) ||
+      !encode_3d(&tv, v_pool, D, P, (uint64_t)dims->num_pages, 64, P, 1))
+    return SEGPAGED_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SEGPAGED_ERR_CUDA;
+  const int sms = device_sm_count(dev);
+  if (sms <= 0) return SEGPAGED_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), st) != cudaSuccess) return SEGPAGED_ERR_CUDA;
+  PrefillParams p;
+  p.page_table = page_table;
+  p.page_table_len = page_table_len;
+  p.units = reinterpret_cast<const int32_t*>(units);
+  p.num_units = (int32_t)num_units;
+  p.counter = static_cast<int32_t*>(workspace);
+  p.status = status;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.total_q = total_q;
+  p.num_q_heads = Hq;
+  p.num_pages = dims->num_pages;
+  p.log2_group = log2_int(G);
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  const int grid = (int)std::min<int64_t>(num_units, sms);
+#define SEGPAGED_LAUNCH(DD, PP) \
+  if (D == DD && P == PP) return launch_prefill<DD, PP>(tq, tk, tv, p, grid, st);
+  SEGPAGED_LAUNCH(128, 16)
+  SEGPAGED_LAUNCH(128, 32)
+  SEGPAGED_LAUNCH(128, 64)
+  SEGPAGED_LAUNCH(128, 128)
+  SEGPAGED_LAUNCH(64, 16)
+  SEGPAGED_LAUNCH(64, 32)
+  SEGPAGED_LAUNCH(64, 64)
+  SEGPAGED_LAUNCH(64, 128)
+#undef SEGPAGED_LAUNCH
+  return SEGPAGED_ERR_DIMS;
+}

@@ -1,0 +1,204 @@
+"""Sets a multi-layer SegPaged prefill workload up on one GPU through the C ABI and runs it.
+
+Per layer: the storage accounting (segpaged_pages_bytes) gives every (sequence, KV head) its stored
+page count, the caller-side page assignment hands out physical ids in one shared pool, segpaged_build
+scatters the layer's dense K/V into the pool (with the RoPE re-alignment when the workload asks for
+it), segpaged_prefill_plan produces the work units, and segpaged_attn_prefill runs the attention.
+Device memory comes from PyTorch; every computation runs in libsegpaged.so.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import segpaged as sp
+from . import synth
+
+
+@dataclass
+class LayerState:
+    cls: np.ndarray            # [B, Hkv, 3]
+    pages_per_head: np.ndarray
+    table: np.ndarray          # int32, physical ids
+    offs: np.ndarray           # int32 [B*Hkv+1]
+    units: np.ndarray | None = None
+    table_dev: torch.Tensor | None = None
+    offs_dev: torch.Tensor | None = None
+    cls_dev: torch.Tensor | None = None
+    units_dev: torch.Tensor | None = None
+    units_host: torch.Tensor | None = None   # pinned staging copy of the plan
+    upload_done: torch.cuda.Event | None = None
+    q: torch.Tensor | None = None
+    o: torch.Tensor | None = None
+    lse: torch.Tensor | None = None
+    stored_bytes: int = 0
+    dense_bytes: int = 0
+
+
+class Runner:
+    """One workload's pools, page tables, plans, queries and outputs on one device.
+
+    shared_dense: all layers scatter the same dense K/V (drawn for layer 0) through their own tables,
+    class maps and queries -- for many-layer workloads whose dense K/V would not fit in memory at once.
+    keep_dense: keep each layer's dense K/V on the device after set-up (tests compare against them).
+    """
+
+    def __init__(self, w: synth.Workload, device="cuda", layers=None, keep_dense=False, page_seed_offset=0,
+                 shared_dense=False):
+        self.w = w
+        self.device = torch.device(device)
+        self.layers = list(range(w.layers)) if layers is None else list(layers)
+        self.keep_dense = keep_dense or shared_dense
+        self.shared_dense = shared_dense
+        self.dense = {}
+        B, H = w.num_seqs, w.num_kv_heads
+        self.dims = sp.Dims(B, w.num_q_heads, H, w.head_dim, w.page_size, 0)
+        self.ctx = np.asarray(w.ctx_lens, np.int32)
+        self.ql = np.asarray(w.q_lens, np.int32)
+        self.state = {}
+        base = 0
+        for li in self.layers:
+            cls = np.ascontiguousarray(w.classes[li], dtype=np.int32)
+            stored, dense, per = sp.segpaged_pages_bytes(self.dims, self.ctx, self.ql, cls)
+            table, offs, n = synth.assign_pages(per.reshape(B, H), w.page_order, seed=w.seed + 7919 * li + page_seed_offset)
+            self.state[li] = LayerState(cls=cls, pages_per_head=per, table=table + base, offs=offs,
+                                        stored_bytes=stored, dense_bytes=dense)
+            base += n
+        self.num_pages = max(base, 1)
+        if w.page_order == "shuffled" and len(self.layers) > 1:   # one permutation over the whole pool
+            perm = np.random.default_rng(w.seed + 104729 + page_seed_offset).permutation(self.num_pages).astype(np.int32)
+            for st in self.state.values():
+                st.table = perm[st.table]
+        self.dims.num_pages = self.num_pages
+        D, P = w.head_dim, w.page_size
+        self.k_pool = torch.empty(self.num_pages, P, D, dtype=torch.bfloat16, device=self.device)
+        self.v_pool = torch.empty(self.num_pages, P, D, dtype=torch.bfloat16, device=self.device)
+        self.cu_k_dev = torch.from_numpy(w.cu_k()).to(self.device)
+        self.ql_dev = torch.from_numpy(self.ql).to(self.device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.workspace = torch.zeros(max(sp.segpaged_prefill_workspace_bytes(0) // 4, 64), dtype=torch.int32,
+                                     device=self.device)
+        self.rope = None
+        if w.rope_theta is not None:
+            self.rope = torch.from_numpy(sp.segpaged_rope_cos_sin(w.rope_theta, w.rope_deltas, D)).to(self.device)
+        self.scale = 1.0 / math.sqrt(D)
+        for li in self.layers:
+            self._setup_layer(li)
+
+    # ------------------------------------------------------------------------------------ set-up
+    def _setup_layer(self, li):
+        w, st = self.w, self.state[li]
+        st.table_dev = torch.from_numpy(st.table).to(self.device)
+        st.offs_dev = torch.from_numpy(st.offs).to(self.device)
+        st.cls_dev = torch.from_numpy(st.cls.reshape(-1)).to(self.device)
+        if self.shared_dense:
+            if not self.dense:
+                _, k, v = synth.layer_inputs(w, 0, device=self.device)
+                self.dense[0] = (k, v)
+            q = synth.layer_inputs(w, li, device=self.device, parts="q")[0]
+        else:
+            q, k, v = synth.layer_inputs(w, li, device=self.device)
+            if self.keep_dense:
+                self.dense[li] = (k, v)
+            else:
+                self._tmp_dense = (k, v)
+        st.q = q
+        st.o = torch.empty_like(q)
+        st.lse = torch.empty(w.num_q_heads, w.total_q, dtype=torch.float32, device=self.device)
+        self.build_layer(li)
+        self._tmp_dense = None
+        self.plan_layer(li)
+        st.units_dev = torch.from_numpy(np.ascontiguousarray(st.units)).to(self.device)
+        st.units_host = torch.from_numpy(np.ascontiguousarray(st.units)).pin_memory()
+
+    def dense_of(self, li):
+        if self._tmp_dense is not None:
+            return self._tmp_dense
+        return self.dense[0 if self.shared_dense else li]
+
+    _tmp_dense = None
+
+    # -------------------------------------------------------------------------------- hot path
+    def account_layer(self, li):
+        """Storage accounting of one layer (host): stored and dense K+V bytes."""
+        st = self.state[li]
+        stored, dense, _ = sp.segpaged_pages_bytes(self.dims, self.ctx, self.ql, st.cls)
+        return stored, dense
+
+    def plan_layer(self, li):
+        """Host planning of one layer's work units (SELECTVISIBLESTATE)."""
+        st = self.state[li]
+        st.units = sp.segpaged_prefill_plan(self.dims, self.ctx, self.ql, st.cls, st.offs)
+        return st.units
+
+    def upload_plan(self, li, stream=None):
+        st = self.state[li]
+        if st.upload_done is not None:
+            st.upload_done.synchronize()     # the previous copy out of the staging buffer has finished
+        st.units_host.numpy()[:] = st.units
+        s = torch.cuda.current_stream(self.device) if stream is None else stream
+        with torch.cuda.stream(s):
+            st.units_dev.copy_(st.units_host, non_blocking=True)
+        st.upload_done = torch.cuda.Event()
+        st.upload_done.record(s)
+
+    def build_layer(self, li, stream=None):
+        k, v = self.dense_of(li)
+        st = self.state[li]
+        sp.segpaged_build(self.dims, k, v, self.cu_k_dev, self.ql_dev, st.cls_dev, st.table_dev, st.offs_dev, self.rope,
+                          self.k_pool, self.v_pool, self.status, stream)
+
+    def prefill(self, li, stream=None):
+        st = self.state[li]
+        sp.segpaged_attn_prefill(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, self.scale,
+                                 st.o, st.lse, self.workspace, self.status, stream)
+
+    def step(self, stream=None):
+        """Prefill of every layer (pools and plans already in place)."""
+        for li in self.layers:
+            self.prefill(li, stream)
+
+    def full_step(self, stream=None, on_prefill=None):
+        """One pass of the whole hot path for every layer: storage accounting and planning on the host,
+        the build scatter and the prefill on the device. on_prefill(li, start) brackets each prefill
+        launch (start=True before, False after) for per-kernel timing."""
+        for li in self.layers:
+            self.account_layer(li)
+            self.plan_layer(li)
+            self.upload_plan(li, stream)
+            self.build_layer(li, stream)
+            if on_prefill:
+                on_prefill(li, True)
+            self.prefill(li, stream)
+            if on_prefill:
+                on_prefill(li, False)
+
+    def check_status(self):
+        s = int(self.status.item())
+        if s:
+            raise RuntimeError(f"device status word {s:#x}")
+
+
+def visible_counts(w: synth.Workload, layer: int, b: int, kh: int) -> np.ndarray:
+    """|V(i)| for every query position of (sequence b, KV head kh) of a layer."""
+    L, Lq = w.ctx_lens[b], w.q_lens[b]
+    i = np.arange(L - Lq, L, dtype=np.int64)
+    g, S, W = (int(x) for x in w.classes[layer, b, kh])
+    if g:
+        return i + 1
+    sink = np.minimum(S, i + 1)
+    lo = np.maximum(i - W + 1, 0)
+    return sink + (i + 1 - lo) - np.clip(sink - lo, 0, None)
+
+
+def visible_flops(w: synth.Workload, layers=None) -> float:
+    """4 * D * sum over (sequence, query head, query row) of |V(i)|: the algorithmic FLOPs of prefill."""
+    total = 0.0
+    for li in (range(w.layers) if layers is None else layers):
+        for b in range(w.num_seqs):
+            for kh in range(w.num_kv_heads):
+                total += 4.0 * w.head_dim * w.group * float(visible_counts(w, li, b, kh).sum())
+    return total

@@ -1,0 +1,188 @@
+"""Python binding of the SegPagedAttention C ABI (include/segpaged.h), with the same names.
+
+Argument marshalling only: torch tensors become raw pointers, numpy arrays become host pointers,
+the current CUDA stream is passed through, and negative return codes raise SegPagedError. Every
+step of the computation runs in libsegpaged.so; if the library is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsegpaged.so")
+UNIT_FIELDS = 16
+
+STATUS_PAGE_ID = 1
+STATUS_TABLE = 2
+STATUS_TIMEOUT = 4
+STATUS_UNIT = 8
+
+# Every function include/segpaged.h declares.
+EXPORTS = ("segpaged_error_string", "segpaged_pages_bytes", "segpaged_rope_cos_sin", "segpaged_build",
+           "segpaged_prefill_plan", "segpaged_prefill_workspace_bytes", "segpaged_attn_prefill")
+
+
+class SegPagedError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {error_string(code)} (code {code})")
+        self.code = code
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+
+
+@dataclass
+class Dims:
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    page_size: int
+    num_pages: int = 0
+
+    def c(self) -> _Dims:
+        return _Dims(self.num_seqs, self.num_q_heads, self.num_kv_heads, self.head_dim, self.page_size, self.num_pages)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libsegpaged.so not built at {LIB_PATH}; run head_sparse_paged_b200/build_ext.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    dp = ctypes.POINTER(_Dims)
+    lib.segpaged_error_string.restype = ctypes.c_char_p
+    lib.segpaged_error_string.argtypes = [ctypes.c_int]
+    lib.segpaged_pages_bytes.restype = i64
+    lib.segpaged_pages_bytes.argtypes = [dp, vp, vp, vp, vp, vp]
+    lib.segpaged_rope_cos_sin.restype = ctypes.c_int
+    lib.segpaged_rope_cos_sin.argtypes = [ctypes.c_double, vp, i32, i32, vp]
+    lib.segpaged_build.restype = ctypes.c_int
+    lib.segpaged_build.argtypes = [dp] + [vp] * 12
+    lib.segpaged_prefill_plan.restype = i64
+    lib.segpaged_prefill_plan.argtypes = [dp, vp, vp, vp, vp, vp, i64]
+    lib.segpaged_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.segpaged_prefill_workspace_bytes.argtypes = [i64]
+    lib.segpaged_attn_prefill.restype = ctypes.c_int
+    lib.segpaged_attn_prefill.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, i64, ctypes.c_float, vp, vp, vp,
+                                          ctypes.c_size_t, vp, vp]
+    return lib
+
+
+_lib = _load()
+
+
+def library():
+    return _lib
+
+
+def error_string(code: int) -> str:
+    return _lib.segpaged_error_string(int(code)).decode()
+
+
+segpaged_error_string = error_string
+
+
+def _host_i32(a, n=None):
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+    if n is not None and a.size != n:
+        raise ValueError(f"expected {n} int32 values, got {a.size}")
+    return a
+
+
+def _hp(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dev(t: torch.Tensor | None, dtype=None, what=""):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{what}: expected a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{what}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def segpaged_pages_bytes(dims: Dims, ctx_len, q_len, cls):
+    """(stored K+V bytes, dense K+V bytes, stored pages per (b, k) as int32 [B*Hkv]). Host only."""
+    B, H = dims.num_seqs, dims.num_kv_heads
+    L, Lq, c = _host_i32(ctx_len, B), _host_i32(q_len, B), _host_i32(cls, B * H * 3)
+    dense = ctypes.c_int64(0)
+    per = np.zeros(B * H, np.int32)
+    r = _lib.segpaged_pages_bytes(ctypes.byref(dims.c()), _hp(L), _hp(Lq), _hp(c), ctypes.byref(dense), _hp(per))
+    if r < 0:
+        raise SegPagedError(int(r), "segpaged_pages_bytes")
+    return int(r), int(dense.value), per
+
+
+def segpaged_rope_cos_sin(theta: float, deltas, head_dim: int) -> np.ndarray:
+    """[B, D/2, 2] float32 (cos, sin) table of delta_b * theta^(-2d/D)."""
+    d = _host_i32(deltas)
+    out = np.zeros((d.size, head_dim // 2, 2), np.float32)
+    r = _lib.segpaged_rope_cos_sin(float(theta), _hp(d), d.size, head_dim, _hp(out))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_rope_cos_sin")
+    return out
+
+
+def segpaged_build(dims: Dims, k_dense, v_dense, cu_seqlens_k, q_len, cls, page_table, page_table_offs,
+                   rope_cos_sin, k_pool, v_pool, status=None, stream=None):
+    """Scatter dense K/V [sum L, Hkv, D] (bf16, CUDA) into k_pool/v_pool [num_pages, P, D]."""
+    bf = torch.bfloat16
+    r = _lib.segpaged_build(ctypes.byref(dims.c()), _dev(k_dense, bf, "k_dense"), _dev(v_dense, bf, "v_dense"),
+                            _dev(cu_seqlens_k, torch.int32, "cu_seqlens_k"), _dev(q_len, torch.int32, "q_len"),
+                            _dev(cls, torch.int32, "cls"), _dev(page_table, torch.int32, "page_table"),
+                            _dev(page_table_offs, torch.int32, "page_table_offs"),
+                            _dev(rope_cos_sin, torch.float32, "rope_cos_sin"), _dev(k_pool, bf, "k_pool"),
+                            _dev(v_pool, bf, "v_pool"), _dev(status, torch.int32, "status"), _stream(stream))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_build")
+
+
+def segpaged_prefill_plan(dims: Dims, ctx_len, q_len, cls, page_table_offs) -> np.ndarray:
+    """Work units (int32 [n, 16], longest first) for segpaged_attn_prefill. Host only."""
+    B, H = dims.num_seqs, dims.num_kv_heads
+    L, Lq = _host_i32(ctx_len, B), _host_i32(q_len, B)
+    c, offs = _host_i32(cls, B * H * 3), _host_i32(page_table_offs, B * H + 1)
+    d = dims.c()
+    n = _lib.segpaged_prefill_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), None, 0)
+    if n < 0:
+        raise SegPagedError(int(n), "segpaged_prefill_plan")
+    units = np.zeros((max(n, 1), UNIT_FIELDS), np.int32)
+    n2 = _lib.segpaged_prefill_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), _hp(units), n)
+    if n2 < 0:
+        raise SegPagedError(int(n2), "segpaged_prefill_plan")
+    return units[:n]
+
+
+def segpaged_prefill_workspace_bytes(num_units: int) -> int:
+    return int(_lib.segpaged_prefill_workspace_bytes(int(num_units)))
+
+
+def segpaged_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, units, softmax_scale, o, lse, workspace,
+                          status=None, stream=None):
+    """O [total_q, Hq, D] bf16 and LSE [Hq, total_q] float32, written in place (CUDA tensors)."""
+    bf = torch.bfloat16
+    n_units = units.shape[0]
+    r = _lib.segpaged_attn_prefill(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]), _dev(k_pool, bf, "k_pool"),
+                                   _dev(v_pool, bf, "v_pool"), _dev(page_table, torch.int32, "page_table"),
+                                   int(page_table.numel()), _dev(units, torch.int32, "units"), int(n_units),
+                                   float(softmax_scale), _dev(o, bf, "o"), _dev(lse, torch.float32, "lse"),
+                                   _dev(workspace, None, "workspace"), int(workspace.numel() * workspace.element_size()),
+                                   _dev(status, torch.int32, "status"), _stream(stream))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_attn_prefill")

@@ -1,0 +1,163 @@
+"""Host-side checks of the C ABI (no GPU): exported symbols, storage accounting, planner, RoPE table and
+argument validation. Expected values come from the oracle (oracle/reference.py)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from head_sparse_paged_b200 import segpaged as sp
+from head_sparse_paged_b200 import synth
+from oracle import reference as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# Work-unit field positions (head_sparse_paged_b200/csrc/plan.h).
+U_QROW, U_POS0, U_NPOS, U_KVH, U_TOFF, U_NSINK, U_W0, U_GLOBAL, U_SINK, U_WIN, U_AN, U_B0, U_BN, U_NTILES, U_TOTAL, U_SEQ = range(16)
+
+
+def test_library_exports_every_declared_symbol():
+    hdr = open(os.path.join(ROOT, "include", "segpaged.h")).read()
+    declared = set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\*?\s+\*?(segpaged_[a-z_]+)\s*\(", hdr, re.M))
+    assert declared == set(sp.EXPORTS), declared
+    lib = ctypes.CDLL(sp.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def _all_layer_cases():
+    out = []
+    for name in ("tiny", "mistral-7b", "llama-3.3-70b", "qwen3-32b"):
+        w = synth.get(name)
+        out.append((name, w, 0))
+    w = synth.dsv4_flash()
+    out += [("dsv4-flash-l0", w, 0), ("dsv4-flash-l3", w, 3)]
+    return out
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_pages_bytes_matches_oracle(case):
+    name, w, layer = _all_layer_cases()[case]
+    dims = sp.Dims(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.page_size)
+    cls = w.classes[layer]
+    stored, dense, per = sp.segpaged_pages_bytes(dims, w.ctx_lens, w.q_lens, cls)
+    o_stored, o_dense, o_per = orc.pages_bytes(w.cu_k(), w.cu_q(), cls[..., 0], cls[..., 1], cls[..., 2], w.page_size, w.head_dim)
+    assert stored == o_stored and dense == o_dense
+    assert per.tolist() == o_per.reshape(-1).tolist()
+
+
+def test_pages_bytes_known_totals():
+    """Stored pages: tiny 16 + 9; Mistral-shaped 128 + 7 x 25; Qwen3-shaped 1024 + 7 x 97; a mixed
+    DeepSeek-style layer 8 x 1024 + 56 x 65 (hand-derived from the storage rule)."""
+    expect = {"tiny": 25, "mistral-7b": 303, "qwen3-32b": 1703, "dsv4-flash-l3": 11832, "dsv4-flash-l0": 65536}
+    for name, w, layer in _all_layer_cases():
+        if name not in expect:
+            continue
+        dims = sp.Dims(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.page_size)
+        _, _, per = sp.segpaged_pages_bytes(dims, w.ctx_lens, w.q_lens, w.classes[layer])
+        assert int(per.sum()) == expect[name], name
+
+
+EDGE = [
+    # (seqs [(L, Lq)], Hq, Hkv, D, P, classes [B][Hkv])
+    ([(256, 64)], 4, 2, 64, 16, [[(1, 0, 0), (0, 4, 64)]]),
+    ([(1000, 300), (37, 37), (5, 0), (129, 1)], 8, 2, 128, 32, [[(0, 0, 100), (1, 0, 0)], [(0, 50, 3), (0, 2, 1)], [(1, 0, 0), (0, 1, 1)], [(0, 128, 1), (1, 0, 0)]]),
+    ([(300, 300)], 8, 8, 64, 128, [[(0, 5, 17), (0, 0, 1), (1, 0, 0), (0, 300, 300), (0, 1000, 2), (0, 64, 64), (0, 127, 129), (0, 3, 250)]]),
+    ([(777, 200)], 16, 2, 128, 16, [[(0, 16, 16), (0, 17, 15)]]),
+    ([(4100, 1030)], 2, 2, 128, 64, [[(0, 64, 1024), (1, 0, 0)]]),
+]
+
+
+def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes):
+    B = len(w_seqs)
+    dims = sp.Dims(B, Hq, Hkv, D, P)
+    ctx = [s[0] for s in w_seqs]
+    ql = [s[1] for s in w_seqs]
+    cls = np.asarray(classes, np.int32)
+    _, _, per = sp.segpaged_pages_bytes(dims, ctx, ql, cls)
+    offs = np.concatenate([[0], np.cumsum(per)]).astype(np.int32)
+    units = sp.segpaged_prefill_plan(dims, ctx, ql, cls, offs)
+    G = Hq // Hkv
+    cu_q = np.concatenate([[0], np.cumsum(ql)])
+    seen = np.zeros((int(cu_q[-1]), Hkv), np.int32)
+    ppt = 128 // P
+    prev = 1 << 30
+    for u in units:
+        assert u[U_NTILES] <= prev  # longest first
+        prev = u[U_NTILES]
+        b, kh = int(u[U_SEQ]), int(u[U_KVH])
+        L, Lq = ctx[b], ql[b]
+        g, S, W = (int(x) for x in cls[b, kh])
+        stored = orc.stored_logical_pages(L, Lq, bool(g), S, W, P)
+        assert u[U_TOTAL] == len(stored) and u[U_TOFF] == offs[b * Hkv + kh]
+        npages = int(u[U_AN] + u[U_BN])
+        assert u[U_NTILES] == -(-npages // ppt)
+        idxs = [x if x < u[U_AN] else int(u[U_B0]) + x - int(u[U_AN]) for x in range(npages)]
+        assert len(set(idxs)) == npages and all(0 <= x < len(stored) for x in idxs)
+        lps = [x if x < u[U_NSINK] else int(u[U_W0]) + x - int(u[U_NSINK]) for x in idxs]
+        assert lps == [stored[x] for x in idxs]          # table index -> logical page is the storage order
+        covered = set()
+        for lp in lps:
+            covered.update(range(lp * P, lp * P + P))
+        assert 1 <= u[U_NPOS] <= 128 // G
+        for r in range(int(u[U_NPOS])):
+            i = int(u[U_POS0]) + r
+            row = int(u[U_QROW]) + r
+            assert row - cu_q[b] == i - (L - Lq)
+            assert set(orc.visible_keys(bool(g), S, W, i).tolist()) <= covered
+            seen[row, kh] += 1
+    assert np.all(seen == 1)
+    return units
+
+
+@pytest.mark.parametrize("case", range(len(EDGE)))
+def test_plan_units_cover_every_row_once_and_every_visible_key(case):
+    _units_cover_exactly(*EDGE[case])
+
+
+@pytest.mark.parametrize("name", ["tiny", "mistral-7b", "llama-3.3-70b", "qwen3-32b"])
+def test_plan_workloads(name):
+    w = synth.get(name)
+    seqs = list(zip(w.ctx_lens, w.q_lens))
+    if name in ("llama-3.3-70b", "qwen3-32b"):       # the set checks are slow in Python at full size
+        seqs = [(min(L, 9000), min(Lq, 700)) for L, Lq in seqs]
+    _units_cover_exactly(seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.page_size, w.classes[0].tolist())
+
+
+def test_rope_table_matches_oracle():
+    deltas = list(range(4096))
+    for D in (64, 128):
+        got = sp.segpaged_rope_cos_sin(1e6, deltas, D)
+        want = orc.rope_cos_sin(1e6, deltas, D)
+        np.testing.assert_array_equal(got, want)
+
+
+def test_validation_errors():
+    dims = sp.Dims(1, 4, 2, 64, 16)
+    with pytest.raises(sp.SegPagedError) as e:
+        sp.segpaged_pages_bytes(sp.Dims(1, 4, 2, 96, 16), [10], [5], [[1, 0, 0], [1, 0, 0]])
+    assert e.value.code == -2
+    with pytest.raises(sp.SegPagedError) as e:
+        sp.segpaged_pages_bytes(sp.Dims(1, 4, 3, 64, 16), [10], [5], [[1, 0, 0]] * 3)
+    assert e.value.code == -2
+    with pytest.raises(sp.SegPagedError) as e:
+        sp.segpaged_pages_bytes(sp.Dims(1, 4, 2, 64, 24), [10], [5], [[1, 0, 0], [1, 0, 0]])
+    assert e.value.code == -2
+    with pytest.raises(sp.SegPagedError) as e:
+        sp.segpaged_pages_bytes(dims, [10], [11], [[1, 0, 0], [1, 0, 0]])
+    assert e.value.code == -4
+    with pytest.raises(sp.SegPagedError) as e:
+        sp.segpaged_pages_bytes(dims, [10], [5], [[1, 0, 0], [0, 4, 0]])
+    assert e.value.code == -3
+    # page-table offsets that disagree with the storage rule
+    with pytest.raises(sp.SegPagedError) as e:
+        sp.segpaged_prefill_plan(dims, [256], [64], [[1, 0, 0], [0, 4, 64]], [0, 16, 24])
+    assert e.value.code == -5
+    lib = sp.library()
+    # NULL dims and NULL arrays
+    assert lib.segpaged_pages_bytes(None, None, None, None, None, None) == -1
+    assert lib.segpaged_attn_prefill(ctypes.byref(dims.c()), None, 1, None, None, None, 0, None, 3, 1.0, None, None,
+                                     None, 256, None, None) == -1
+    assert lib.segpaged_build(ctypes.byref(dims.c()), *([None] * 12)) == -1
+    assert sp.error_string(-5).startswith("page-table")
