@@ -352,3 +352,64 @@ extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, i
 #undef SEGPAGED_LAUNCH
   return SEGPAGED_ERR_DIMS;
 }
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free prefill entry point.
+//
+// Some callers cannot allocate device memory when they run prefill -- for example code running under
+// a framework's own memory pool, or a runtime that forbids allocation on its request path -- so they
+// cannot provide the work-unit list and the work-counter workspace that segpaged_attn_prefill needs.
+// For them, both live in one file-scope device array below. Every GPU that loads this library holds
+// it (2 MiB) until the process exits. All calls on a device share it and it keeps the last call's
+// contents, so the counter is cleared on every call; calls whose work overlaps on the GPU race on it.
+// ------------------------------------------------------------------------------------------------
+namespace {
+constexpr int64_t kNoAllocMaxUnits = 32768;   // the most work units one call accepts
+constexpr int64_t kNoAllocUnitOffset = 64;    // int32 words before the unit list (counter in word 0)
+}  // namespace
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocUnitOffset + kNoAllocMaxUnits * U_NFIELDS];
+
+namespace {
+std::mutex g_noalloc_mutex;
+int32_t* g_noalloc_addr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array on the current device. In host code the array's name is only a
+// host-side stand-in, so its address is looked up once per device, with that device current.
+int noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SEGPAGED_ERR_CUDA;
+    g_noalloc_addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return SEGPAGED_OK;
+}
+}  // namespace
+
+extern "C" int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const void* q, int32_t total_q,
+                                             const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                             int64_t page_table_len, const segpaged_unit* units_host,
+                                             int64_t num_units, float softmax_scale, void* o, float* lse,
+                                             int32_t* status, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (num_units < 0) return SEGPAGED_ERR_DIMS;
+  if (num_units > kNoAllocMaxUnits) return SEGPAGED_ERR_CAPACITY;
+  if (num_units == 0) return SEGPAGED_OK;
+  if (!units_host) return SEGPAGED_ERR_NULL;
+  int32_t* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  int32_t* units_dev = scratch + kNoAllocUnitOffset;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(units_dev, units_host, sizeof(segpaged_unit) * (size_t)num_units, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return SEGPAGED_ERR_CUDA;
+  // The work counter (word 0) is zeroed on the stream by segpaged_attn_prefill before its launch.
+  return segpaged_attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len,
+                               reinterpret_cast<const segpaged_unit*>(units_dev), num_units, softmax_scale, o, lse,
+                               scratch, kNoAllocUnitOffset * sizeof(int32_t), status, stream);
+}

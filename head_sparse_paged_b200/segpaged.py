@@ -24,7 +24,8 @@ STATUS_UNIT = 8
 
 # Every function include/segpaged.h declares.
 EXPORTS = ("segpaged_error_string", "segpaged_pages_bytes", "segpaged_rope_cos_sin", "segpaged_build",
-           "segpaged_prefill_plan", "segpaged_prefill_workspace_bytes", "segpaged_attn_prefill")
+           "segpaged_prefill_plan", "segpaged_prefill_workspace_bytes", "segpaged_attn_prefill",
+           "segpaged_attn_prefill_noalloc")
 
 
 class SegPagedError(RuntimeError):
@@ -72,6 +73,8 @@ def _load():
     lib.segpaged_attn_prefill.restype = ctypes.c_int
     lib.segpaged_attn_prefill.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, i64, ctypes.c_float, vp, vp, vp,
                                           ctypes.c_size_t, vp, vp]
+    lib.segpaged_attn_prefill_noalloc.restype = ctypes.c_int
+    lib.segpaged_attn_prefill_noalloc.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, i64, ctypes.c_float, vp, vp, vp, vp]
     return lib
 
 
@@ -186,3 +189,23 @@ def segpaged_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, units, soft
                                    _dev(status, torch.int32, "status"), _stream(stream))
     if r < 0:
         raise SegPagedError(r, "segpaged_attn_prefill")
+
+
+NOALLOC_MAX_UNITS = 32768
+
+
+def segpaged_attn_prefill_noalloc(dims: Dims, q, k_pool, v_pool, page_table, units_host, softmax_scale, o, lse,
+                                  status=None, stream=None):
+    """segpaged_attn_prefill for callers that cannot allocate device memory: the plan comes straight from
+    the host (int32 [n, 16] from segpaged_prefill_plan) and the library's own static device array holds
+    it and the work counter. At most NOALLOC_MAX_UNITS units; calls that overlap on the GPU race."""
+    bf = torch.bfloat16
+    units = np.ascontiguousarray(np.asarray(units_host, dtype=np.int32).reshape(-1, UNIT_FIELDS))
+    r = _lib.segpaged_attn_prefill_noalloc(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]),
+                                           _dev(k_pool, bf, "k_pool"), _dev(v_pool, bf, "v_pool"),
+                                           _dev(page_table, torch.int32, "page_table"), int(page_table.numel()),
+                                           _hp(units), int(units.shape[0]), float(softmax_scale), _dev(o, bf, "o"),
+                                           _dev(lse, torch.float32, "lse"), _dev(status, torch.int32, "status"),
+                                           _stream(stream))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_attn_prefill_noalloc")

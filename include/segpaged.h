@@ -173,6 +173,28 @@ int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t tota
                           float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
                           int32_t* status, void* stream);
 
+/*
+ * segpaged_attn_prefill without caller-provided device scratch. The paper has no counterpart: this
+ * entry point exists for callers that cannot allocate device memory when they run prefill (for
+ * example code inside a framework's own memory pool, or a runtime that forbids allocation on its
+ * request path), so they cannot provide the unit list and workspace segpaged_attn_prefill needs.
+ * It computes the same result from the same arguments, except:
+ *   units_host (host) [num_units] straight from segpaged_prefill_plan; it is copied on `stream` into a
+ *     library-owned device array, so keep it unchanged until the stream has passed this call
+ *     (a pageable buffer is staged before the call returns);
+ *   no workspace arguments.
+ * The library-owned array is a static device array of 2 MiB that every GPU loading the library keeps
+ * until the process exits; it holds at most 32768 units (more return SEGPAGED_ERR_CAPACITY). The
+ * first call on a device looks up the array's device address; make that first call before any
+ * stream capture. Every call on a device shares the array and it keeps the last call's contents (the
+ * work counter is cleared on every call): calls whose work overlaps on the GPU race, so serialise
+ * them (one stream, or events). Allocates no memory.
+ */
+int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
+                                  const void* v_pool, const int32_t* page_table, int64_t page_table_len,
+                                  const segpaged_unit* units_host, int64_t num_units, float softmax_scale, void* o,
+                                  float* lse, int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
