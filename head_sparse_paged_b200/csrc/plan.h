@@ -47,15 +47,15 @@ SP_HD Split storage_split(int32_t L, int32_t Lq, int32_t is_global, int32_t sink
   return s;
 }
 
-// Work unit: one (sequence, KV head) and a tile of up to 128/G consecutive query positions, all G
-// query heads of the group (128 rows of the tensor-core tile). Its keys are the pages at list
+// Work unit: one (sequence, KV head) and up to 2 x 128/G consecutive query positions, all G query heads
+// of the group: two 128-row tensor-core tiles that share every K/V tile. Its keys are the pages at list
 // positions [0, a_n + b_n): list position x < a_n is table index x (sink part), list position
 // x >= a_n is table index b0 + (x - a_n) (window part). KV tiles are groups of 128/P consecutive
 // list positions; n_tiles = ceil((a_n + b_n) / (128/P)).
 enum UnitField {
   U_QROW = 0,   // row of the first position in Q / O (index into the packed query rows)
   U_POS0 = 1,   // absolute position of the first row
-  U_NPOS = 2,   // valid positions in this tile (<= 128/G)
+  U_NPOS = 2,   // valid positions in this unit (<= 2 x 128/G)
   U_KVH = 3,    // KV head
   U_TOFF = 4,   // offset of the head's page table
   U_NSINK = 5,  // Split::n_sink

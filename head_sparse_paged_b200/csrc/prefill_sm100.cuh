@@ -5,20 +5,25 @@
 // storage removing the attn_mask penalty). Visibility: key j is visible to query position i iff
 // j <= i and (global head, or j < S, or j > i - W).
 //
-// Work: units of (sequence, KV head, up to 128/G query positions x G query heads = 128 tile rows),
-// planned on the host with their visible page ranges and sorted longest-first; CTAs (one per SM)
-// claim them through a global atomic counter.
+// Work: units of (sequence, KV head, up to 2 x 128/G query positions x G query heads), planned on the
+// host with their visible page ranges and sorted longest-first; CTAs (one per SM) claim them through a
+// global atomic counter. A unit is two 128-row query tiles that share every K/V tile of the unit.
 //
-// Per CTA, 6 warps:
-//   warp 0   producer: claims units, TMA-loads the Q tile (3-D map over [rows, Hq, D], box 64 x G x
-//            128/G) and, for every 128-key tile, the K and V pages (3-D map over [pages, P, D],
-//            coordinate = physical page id) into 128B-swizzled shared-memory slots.
-//   warp 1   MMA issuer: S = Q K^T (tcgen05.mma, both operands from shared memory, f32 in TMEM,
-//            double-buffered) and O += P V (P read from TMEM, V MN-major from shared memory).
-//   warps 2-5 softmax: one tile row per thread. tcgen05.ld of the S row, per-row bounds only on
-//            edge tiles, row max, lazy O rescale (only when the running max grows by more than
-//            2^8), exp2, row sum, P written back to TMEM as bf16 over the S buffer, and the
-//            epilogue (O / l -> bf16, LSE = ln 2 * (m + log2 l)).
+// Per CTA, 12 warps (3 warpgroups):
+//   warps 0-3   softmax for query tile 0, warps 4-7 softmax for query tile 1: one tile row per thread.
+//               tcgen05.ld of the S row, per-row bounds only on edge tiles, row max (3-input max),
+//               lazy O rescale (only when the running max grows by more than 2^8), exp2 -- three of
+//               every four element pairs on the MUFU unit, the fourth on the FMA pipe by a cubic --,
+//               row sum and scaling in packed f32x2 arithmetic, P written back to TMEM as bf16 over S,
+//               and the epilogue (O / l -> bf16, LSE = ln 2 * (m + log2 l)).
+//   warp 8      producer: claims units, TMA-loads both Q tiles (3-D map over [rows, Hq, D], box
+//               64 x G x 128/G) and, for every 128-key tile, the K and V pages (3-D map over
+//               [pages, P, D], coordinate = physical page id) into 128B-swizzled shared-memory slots.
+//   warp 9      MMA issuer, in the order PV0(j-1), S0(j), PV1(j-1), S1(j): S_t = Q_t K^T
+//               (tcgen05.mma, both operands in shared memory, f32 in TMEM) and O_t += P_t V (P from
+//               TMEM, V MN-major from shared memory). The commit that publishes S_t(j) also covers
+//               PV_t(j-1), so when a softmax warp sees S_t(j) its O_t is stable and can be rescaled.
+//   warps 10-11 idle.
 // Every wait is bounded: on a timeout the CTA raises its abort flag, reports
 // SEGPAGED_STATUS_TIMEOUT, drains the MMA pipe and frees its tensor memory before returning.
 #pragma once
@@ -37,19 +42,24 @@ constexpr int32_t kStatusUnit = 8;
 
 template <int D, int P>
 struct PrefillCfg {
-  static constexpr int BM = 128;                 // tile rows (positions x heads)
+  static constexpr int BM = 128;                 // rows of one query tile (positions x heads)
   static constexpr int BN = 128;                 // keys per KV tile
   static constexpr int NH = D / 64;              // 128-byte swizzle column blocks across D
   static constexpr int BLK = BN * 128;           // bytes of one 64-column block of a 128-row tile
   static constexpr int TILE_BYTES = BN * D * 2;  // one K or V tile
-  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int Q_BYTES = BM * D * 2;     // one query tile
   static constexpr int NSLOT = (D == 128) ? 5 : 10;
   static constexpr int PPT = BN / P;             // pages per KV tile
   static constexpr int SMEM_BYTES = 2 * Q_BYTES + NSLOT * TILE_BYTES + 1024;
-  static constexpr int THREADS = 192;
-  static constexpr uint32_t TMEM_COLS = 512;     // S0 [0,128) S1 [128,256) O [256, 256+D)
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t TMEM_COLS = 512;     // S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D)
   static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t IDESC_O = ptx::idesc_bf16_f32(128, D, 0, 1);
+  // Register split (setmaxnreg): 256 softmax threads x 208 + 128 other threads x 80 = 63488, within the
+  // 384 x 168 = 64512 registers the block is launched with.
+  static constexpr int REGS_SOFTMAX = 208;
+  static constexpr int REGS_OTHER = 80;
+  static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= 384 * 168, "register split exceeds the launch budget");
 };
 
 struct PrefillParams {
@@ -67,9 +77,9 @@ struct PrefillParams {
 
 struct PrefillShared {
   uint64_t unit_full[2], unit_empty[2];
-  uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[2], p_full[2], pv_done[2];
-  uint64_t o_free, mma_drain;
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+  uint64_t mma_drain;
   uint64_t kv_full[10], kv_empty[10];
   __align__(16) int32_t unit[2][U_NFIELDS];
   uint32_t tmem_base;
@@ -85,15 +95,72 @@ __device__ __forceinline__ int32_t unit_logical_page(const int32_t* u, int32_t i
   return idx < u[U_NSINK] ? idx : u[U_W0] + (idx - u[U_NSINK]);
 }
 
+// ----------------------------------------------------------------------------- packed f32 math
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair, on the FMA and integer pipes: n = round(x) through the 1.5 * 2^23 rounding trick,
+// f = x - n in [-1/2, 1/2], 2^f by a cubic minimising relative error (coefficients from
+// csrc/fit_exp2_poly.py, max relative error 7.5e-5), then n is added to the exponent bits. x is
+// clamped to >= -126 so the exponent never wraps; masked logits (-inf) then give ~1e-38 instead of 0.
+__device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t nmagic = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t t = f2_add(xc, magic);                  // low mantissa bits hold round(x)
+  const uint64_t n = f2_add(t, nmagic);                  // round(x) as a float
+  const uint64_t neg1 = f2_pack(-1.0f, -1.0f);
+  const uint64_t f = f2_fma(n, neg1, xc);                // x - round(x)
+  uint64_t p = f2_fma(f2_pack(0x1.c3f76p-5f, 0x1.c3f76p-5f), f, f2_pack(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+  p = f2_fma(p, f, f2_pack(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+  p = f2_fma(p, f, f2_pack(0x1.fff692p-1f, 0x1.fff692p-1f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
 template <int D, int P>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
     segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
   using C = PrefillCfg<D, P>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ PrefillShared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                        // 2 x Q_BYTES
+  uint8_t* sQ = smem;                        // 2 query tiles x Q_BYTES
   uint8_t* sKV = smem + 2 * C::Q_BYTES;      // NSLOT x TILE_BYTES
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &sh.abort;
@@ -103,14 +170,14 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sh.unit_full[i], 1);
-      ptx::mbar_init(&sh.unit_empty[i], 5);   // MMA lane 0 + 4 softmax warps
-      ptx::mbar_init(&sh.q_full[i], 1);
-      ptx::mbar_init(&sh.q_empty[i], 1);
+      ptx::mbar_init(&sh.unit_empty[i], 9);   // MMA lane 0 + 8 softmax warps
       ptx::mbar_init(&sh.s_full[i], 1);
       ptx::mbar_init(&sh.p_full[i], 4);
-      ptx::mbar_init(&sh.pv_done[i], 1);
+      ptx::mbar_init(&sh.o_full[i], 1);
+      ptx::mbar_init(&sh.o_free[i], 4);
     }
-    ptx::mbar_init(&sh.o_free, 4);
+    ptx::mbar_init(&sh.q_full, 1);
+    ptx::mbar_init(&sh.q_empty, 1);
     ptx::mbar_init(&sh.mma_drain, 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       ptx::mbar_init(&sh.kv_full[i], 1);
@@ -119,17 +186,17 @@ __global__ void __launch_bounds__(192, 1)
     sh.abort = 0;
     ptx::mbar_fence_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     ptx::tma_prefetch_desc(&tm_q);
     ptx::tma_prefetch_desc(&tm_k);
     ptx::tma_prefetch_desc(&tm_v);
   }
-  if (warp == 1) {
+  if (warp == 9) {
     ptx::tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
   // KV slots start zeroed: a partial tile leaves earlier (finite) data in the rows it does not
-  // load, and those columns are masked, so their probability is exactly 0.
+  // load, and those columns are masked.
   for (int x = threadIdx.x; x < C::NSLOT * C::TILE_BYTES / 16; x += blockDim.x)
     reinterpret_cast<uint4*>(sKV)[x] = make_uint4(0, 0, 0, 0);
   ptx::fence_proxy_async_smem();
@@ -137,17 +204,19 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  const uint32_t tS = tmem, tO = tmem + 256;
   const int G = 1 << p.log2_group;
+  const int npos = C::BM >> p.log2_group;    // positions per query tile
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t kv_item = 0, qcnt = 0;
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------------------------- producer
+      uint32_t kv_item = 0;
       for (uint32_t ring = 0;; ++ring) {
-        const int32_t u = atomicAdd(p.counter, 1);
         const int slot = ring & 1;
         if (!ptx::mbar_wait(&sh.unit_empty[slot], ((ring >> 1) & 1) ^ 1, abort, status, kStatusTimeout)) break;
+        // claim the next unit only once a ring slot is free, so no CTA sits on work it cannot start
+        const int32_t u = atomicAdd(p.counter, 1);
         const bool done = u >= p.num_units;
         int32_t* U = sh.unit[slot];
         if (done) {
@@ -159,23 +228,25 @@ __global__ void __launch_bounds__(192, 1)
         }
         ptx::mbar_arrive(&sh.unit_full[slot]);
         if (done) break;
-        const int qb = qcnt & 1;
-        if (!ptx::mbar_wait(&sh.q_empty[qb], ((qcnt >> 1) & 1) ^ 1, abort, status, kStatusTimeout)) break;
-        ptx::mbar_arrive_expect_tx(&sh.q_full[qb], C::Q_BYTES);
+        // both query tiles: the unit's positions [0, npos) and [npos, 2 npos)
+        if (!ptx::mbar_wait(&sh.q_empty, (ring & 1) ^ 1, abort, status, kStatusTimeout)) break;
+        ptx::mbar_arrive_expect_tx(&sh.q_full, 2 * C::Q_BYTES);
 #pragma unroll
-        for (int h = 0; h < C::NH; ++h)
-          ptx::tma_load_3d(sQ + qb * C::Q_BYTES + h * C::BLK, &tm_q, h * 64, U[U_KVH] * G, U[U_QROW], &sh.q_full[qb]);
-        ++qcnt;
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int h = 0; h < C::NH; ++h)
+            ptx::tma_load_3d(sQ + t * C::Q_BYTES + h * C::BLK, &tm_q, h * 64, U[U_KVH] * G, U[U_QROW] + t * npos,
+                             &sh.q_full);
         const int32_t npages = U[U_AN] + U[U_BN];
         const int32_t ntiles = U[U_NTILES];
         const int64_t toff = U[U_TOFF];
         bool ok = true;
-        for (int32_t t = 0; t < ntiles && ok; ++t) {
+        for (int32_t j = 0; j < ntiles && ok; ++j) {
           int32_t pages[C::PPT];
           int32_t n_ok = 0;
 #pragma unroll
           for (int c = 0; c < C::PPT; ++c) {
-            const int32_t x = t * C::PPT + c;
+            const int32_t x = j * C::PPT + c;
             pages[c] = -1;
             if (x < npages) {
               const int32_t idx = unit_table_index(U, x);
@@ -194,7 +265,7 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
 #pragma unroll
-          for (int which = 0; which < 2; ++which) {
+          for (int which = 0; which < 2; ++which) {  // K then V
             const int s = kv_item % C::NSLOT;
             if (!ptx::mbar_wait(&sh.kv_empty[s], ((kv_item / C::NSLOT) & 1) ^ 1, abort, status, kStatusTimeout)) {
               ok = false;
@@ -215,30 +286,40 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (!ok) break;
       }
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    } else if (warp == 9 && lane == 0) {
+      // -------------------------------------------------------------------------- MMA issuer
       const uint32_t q_base = ptx::smem_addr(sQ), kv_base = ptx::smem_addr(sKV);
-      uint32_t g = 0, kv_item = 0, ucnt = 0;
-      bool prev_valid = false, prev_first = false;
-      uint32_t prev_g = 0, prev_vi = 0, prev_ucnt = 0;
+      uint32_t kv_item = 0, ucnt = 0, pcount[2] = {0, 0};
       bool ok = true;
-      auto issue_pv = [&](uint32_t pg, uint32_t vi, bool first, uint32_t pu) -> bool {
-        if (!ptx::mbar_wait(&sh.p_full[pg & 1], (pg >> 1) & 1, abort, status, kStatusTimeout)) return false;
-        if (first && pu > 0 && !ptx::mbar_wait(&sh.o_free, (pu - 1) & 1, abort, status, kStatusTimeout)) return false;
+      // O_t (+)= P_t V for the V tile in KV item vi; `first` starts the unit's accumulation.
+      auto issue_pv = [&](int t, uint32_t vi, bool first) -> bool {
+        if (!ptx::mbar_wait(&sh.p_full[t], pcount[t] & 1, abort, status, kStatusTimeout)) return false;
+        ++pcount[t];
+        if (first && ucnt > 0 && !ptx::mbar_wait(&sh.o_free[t], (ucnt - 1) & 1, abort, status, kStatusTimeout))
+          return false;
         const int s = vi % C::NSLOT;
-        if (!ptx::mbar_wait(&sh.kv_full[s], (vi / C::NSLOT) & 1, abort, status, kStatusTimeout)) return false;
+        if (t == 0 && !ptx::mbar_wait(&sh.kv_full[s], (vi / C::NSLOT) & 1, abort, status, kStatusTimeout))
+          return false;
         ptx::tc_fence_after();
-        const uint32_t pa = tS + (pg & 1) * 128;
+        const uint32_t pa = tmem + t * 128;                 // P_t: bf16 pairs over the first 64 columns of S_t
+        const uint32_t od = tmem + 256 + t * D;
         const uint32_t vb = kv_base + s * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          ptx::umma_ts(tO, pa + kk * 8, ptx::sw128_desc(vb + kk * 16 * 128, C::BLK, 1024), C::IDESC_O,
+          ptx::umma_ts(od, pa + kk * 8, ptx::sw128_desc(vb + kk * 16 * 128, C::BLK, 1024), C::IDESC_O,
                        (kk > 0 || !first) ? 1u : 0u);
-        ptx::umma_commit(&sh.pv_done[pg & 1]);
-        ptx::umma_commit(&sh.kv_empty[s]);
         return true;
+      };
+      auto issue_s = [&](int t, uint32_t kb) {
+        const uint32_t qa = q_base + t * C::Q_BYTES;
+        const uint32_t sd = tmem + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
+          ptx::umma_ss(sd, ptx::sw128_desc(qa + off, 16, 1024), ptx::sw128_desc(kb + off, 16, 1024), C::IDESC_S,
+                       kk > 0 ? 1u : 0u);
+        }
+        ptx::umma_commit(&sh.s_full[t]);
       };
       for (uint32_t ring = 0; ok; ++ring) {
         const int slot = ring & 1;
@@ -246,75 +327,68 @@ __global__ void __launch_bounds__(192, 1)
         const int32_t ntiles = sh.unit[slot][U_NTILES];
         ptx::mbar_arrive(&sh.unit_empty[slot]);
         if (ntiles < 0) break;
-        const int qb = ucnt & 1;
-        if (!ptx::mbar_wait(&sh.q_full[qb], (ucnt >> 1) & 1, abort, status, kStatusTimeout)) { ok = false; break; }
-        const uint32_t qa = q_base + qb * C::Q_BYTES;
-        for (int32_t t = 0; t < ntiles; ++t) {
+        if (!ptx::mbar_wait(&sh.q_full, ucnt & 1, abort, status, kStatusTimeout)) { ok = false; break; }
+        uint32_t prev_vi = 0;
+        for (int32_t j = 0; j < ntiles && ok; ++j) {
           const uint32_t ki = kv_item, vi = kv_item + 1;
           kv_item += 2;
+          if (j > 0 && !issue_pv(0, prev_vi, j == 1)) { ok = false; break; }
           const int s = ki % C::NSLOT;
           if (!ptx::mbar_wait(&sh.kv_full[s], (ki / C::NSLOT) & 1, abort, status, kStatusTimeout)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t kb = kv_base + s * C::TILE_BYTES;
-          const uint32_t sd = tS + (g & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-            ptx::umma_ss(sd, ptx::sw128_desc(qa + off, 16, 1024), ptx::sw128_desc(kb + off, 16, 1024), C::IDESC_S,
-                         kk > 0 ? 1u : 0u);
+          issue_s(0, kb);
+          if (j > 0) {
+            if (!issue_pv(1, prev_vi, j == 1)) { ok = false; break; }
+            ptx::umma_commit(&sh.kv_empty[prev_vi % C::NSLOT]);
           }
-          ptx::umma_commit(&sh.s_full[g & 1]);
+          issue_s(1, kb);
           ptx::umma_commit(&sh.kv_empty[s]);
-          if (t == ntiles - 1) ptx::umma_commit(&sh.q_empty[qb]);
-          if (prev_valid && !issue_pv(prev_g, prev_vi, prev_first, prev_ucnt)) { ok = false; break; }
-          prev_valid = true;
-          prev_g = g;
+          if (j == ntiles - 1) ptx::umma_commit(&sh.q_empty);
           prev_vi = vi;
-          prev_first = (t == 0);
-          prev_ucnt = ucnt;
-          ++g;
         }
+        if (!ok) break;
+        // the unit's last PV of each tile publishes its O
+        if (!issue_pv(0, prev_vi, ntiles == 1)) break;
+        ptx::umma_commit(&sh.o_full[0]);
+        if (!issue_pv(1, prev_vi, ntiles == 1)) break;
+        ptx::umma_commit(&sh.o_full[1]);
+        ptx::umma_commit(&sh.kv_empty[prev_vi % C::NSLOT]);
         ++ucnt;
       }
-      if (ok && prev_valid) issue_pv(prev_g, prev_vi, prev_first, prev_ucnt);
       // Drain: every MMA this CTA issued has completed before tensor memory is released.
       ptx::umma_commit(&sh.mma_drain);
       ptx::mbar_wait(&sh.mma_drain, 0, abort, status, kStatusTimeout);
     }
-    __syncwarp();
   } else {
-    // ---------------------------------------------------------------------- softmax warps 2..5
-    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int tile = warp >> 2;       // query tile of this warpgroup
+    const int quarter = warp & 3;     // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t sbuf = tmem + tile * 128 + lane_off;
+    const uint32_t obuf = tmem + 256 + tile * D + lane_off;
     const float sl2 = p.scale_log2;
-    uint32_t g = 0, pv_seen0 = 0, pv_seen1 = 0;
-    bool ok = true;
+    const uint64_t sl2_2 = f2_pack(sl2, sl2);
+    uint32_t scount = 0, ucnt = 0;
     // The tcgen05.ld/st below are warp-collective, so every wait's outcome is made warp-uniform.
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kStatusTimeout));
     };
-    // Waits until PV number k has completed. Completions of pv_done[k & 1] are observed strictly in
-    // order, and at most one of them is ever pending when this runs, so parity tracking is exact.
-    auto wait_pv = [&](uint32_t k) -> bool {
-      uint32_t& seen = (k & 1) ? pv_seen1 : pv_seen0;
-      while (seen <= (k >> 1)) {
-        if (!wwait(&sh.pv_done[k & 1], seen & 1)) return false;
-        ++seen;
-      }
-      return true;
-    };
-    for (uint32_t ring = 0; ok; ++ring) {
+    for (uint32_t ring = 0;; ++ring) {
       const int slot = ring & 1;
       if (!wwait(&sh.unit_full[slot], (ring >> 1) & 1)) break;
-      int32_t u[U_NFIELDS];
-#pragma unroll
-      for (int i = 0; i < U_NFIELDS; ++i) u[i] = sh.unit[slot][i];
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
+      // The descriptor stays in shared memory while this unit runs: the slot is released only after
+      // the epilogue, and the producer refills a slot only once every consumer has released it.
+      const int32_t* u = sh.unit[slot];
       const int32_t ntiles = u[U_NTILES];
-      if (ntiles < 0) break;
-      const int32_t pslot = row >> p.log2_group;
+      if (ntiles < 0) {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
+        break;
+      }
+      const int32_t pslot = tile * npos + (row >> p.log2_group);
       const bool valid_row = pslot < u[U_NPOS];
       const int32_t i_pos = u[U_POS0] + (valid_row ? pslot : u[U_NPOS] - 1);
       const int32_t head = u[U_KVH] * G + (row & (G - 1));
@@ -322,23 +396,24 @@ __global__ void __launch_bounds__(192, 1)
       const int32_t S = u[U_SINK], W = u[U_WIN];
       const int32_t npages = u[U_AN] + u[U_BN];
       float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
 
-      for (int32_t t = 0; t < ntiles; ++t, ++g) {
-        if (!wwait(&sh.s_full[g & 1], (g >> 1) & 1)) { ok = false; break; }
+      for (int32_t j = 0; j < ntiles; ++j) {
+        if (!wwait(&sh.s_full[tile], scount & 1)) { ok = false; break; }
+        ++scount;
         ptx::tc_fence_after();
-        const uint32_t sbuf = tS + (g & 1) * 128 + lane_off;
         float s[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c) ptx::tmem_ld32(sbuf + c * 32, reinterpret_cast<uint32_t*>(s) + c * 32);
         ptx::tmem_ld_wait();
 
-        // Logical page of every slot of this tile; a row needs per-column bounds only if some key of
-        // the tile is invisible to it (causal edge, window edge, sink tail, or a short last tile).
+        // Logical page of every slot of this KV tile; a row needs per-column bounds only if some key
+        // of the tile is invisible to it (causal edge, window edge, sink tail, or a short last tile).
         int32_t lp[C::PPT];
         bool need_mask = false;
 #pragma unroll
         for (int c = 0; c < C::PPT; ++c) {
-          const int32_t x = t * C::PPT + c;
+          const int32_t x = j * C::PPT + c;
           if (x < npages) {
             lp[c] = unit_logical_page(u, unit_table_index(u, x));
             const int32_t j0 = lp[c] * P, j1 = j0 + P - 1;
@@ -352,77 +427,96 @@ __global__ void __launch_bounds__(192, 1)
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < C::PPT; ++c) {
+            const int32_t base = lp[c] * P;
 #pragma unroll
             for (int r = 0; r < P; ++r) {
-              const int32_t j = lp[c] * P + r;
-              const bool vis = lp[c] >= 0 && j <= i_pos && (is_global || j < S || j > i_pos - W);
+              const int32_t jj = base + r;
+              const bool vis = lp[c] >= 0 && jj <= i_pos && (is_global || jj < S || jj > i_pos - W);
               if (!vis) s[c * P + r] = -INFINITY;
             }
           }
         }
-        float mx = s[0];
+        float mx = fmax3(s[0], s[1], s[2]);
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 3; c < 127; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
+        mx = fmaxf(mx, s[127]);
         const float m_tile = mx * sl2;
-
-        if (g >= 2 && !wait_pv(g - 2)) { ok = false; break; }
         const float m_new = fmaxf(m_run, m_tile);
         bool resc = false;
-        if (t == 0) {
+        if (j == 0) {
           m_run = m_new;
         } else {
           resc = m_new > m_run + 8.0f;
         }
-        if (__any_sync(0xffffffffu, resc)) {
-          // O must hold every PV issued so far before it is rescaled in place.
-          if (!wait_pv(g - 1)) { ok = false; break; }
-          ptx::tc_fence_after();
-          const float alpha = resc ? ptx::ex2(m_run - m_new) : 1.0f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tO + lane_off + c * 32, r);
-            ptx::tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-            ptx::tmem_st32(tO + lane_off + c * 32, r);
-          }
-          ptx::tmem_st_wait();
-          if (resc) {
-            l_run *= alpha;
-            m_run = m_new;
-          }
+        const float alpha = resc ? ptx::ex2(m_run - m_new) : 1.0f;
+        if (resc) {
+          l_run *= alpha;
+          m_run = m_new;
         }
         const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-        float rs = 0.f;
-        uint32_t pk[64];
+        const uint64_t nmu2 = f2_pack(-mu, -mu);
+        uint64_t sum2 = f2_pack(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = ptx::ex2(fmaf(s[2 * c], sl2, -mu));
-          const float p1 = ptx::ex2(fmaf(s[2 * c + 1], sl2, -mu));
-          rs += p0 + p1;
-          pk[c] = ptx::pack_bf16x2(p0, p1);
+        for (int h = 0; h < 2; ++h) {          // two halves of 64 columns -> 32 packed P columns each
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int e = h * 64 + 2 * c;
+            const uint64_t x2 = f2_fma(f2_pack(s[e], s[e + 1]), sl2_2, nmu2);
+            uint64_t p2;
+            if ((c & 3) == 3) {
+              p2 = exp2_poly_pair(x2);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p2 = f2_pack(ptx::ex2(x0), ptx::ex2(x1));
+            }
+            sum2 = f2_add(sum2, p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            pk[c] = ptx::pack_bf16x2(p0, p1);
+          }
+          ptx::tmem_st32(sbuf + h * 32, pk);
         }
-        l_run += rs;
-        ptx::tmem_st32(sbuf, pk);
-        ptx::tmem_st32(sbuf + 32, pk + 32);
+        if (__any_sync(0xffffffffu, resc)) {
+          // Rescale O_t in place now that S is dead. O_t holds every PV issued so far (the commit that
+          // published S_t(j) covered PV_t(j-1)), and PV_t(j) waits for this warp's p_full arrival.
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(obuf + c * 32, r);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              float lo, hi;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), a2), lo, hi);
+              r[2 * k] = __float_as_uint(lo);
+              r[2 * k + 1] = __float_as_uint(hi);
+            }
+            ptx::tmem_st32(obuf + c * 32, r);
+          }
+        }
+        float sa, sb;
+        f2_unpack(sum2, sa, sb);
+        l_run += sa + sb;
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.p_full[g & 1]);
+        if (lane == 0) ptx::mbar_arrive(&sh.p_full[tile]);
       }
       if (!ok) break;
 
       // ------------------------------------------------------------------------------ epilogue
-      if (!wait_pv(g - 1)) break;
+      if (!wwait(&sh.o_full[tile], ucnt & 1)) break;
       ptx::tc_fence_after();
       const float inv_l = 1.0f / l_run;
       const int64_t qrow = (int64_t)u[U_QROW] + pslot;
       __nv_bfloat16* orow = p.o + (qrow * p.num_q_heads + head) * D;
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        ptx::tmem_ld32(tO + lane_off + c * 32, r);
+        ptx::tmem_ld32(obuf + c * 32, r);
         ptx::tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
@@ -437,14 +531,18 @@ __global__ void __launch_bounds__(192, 1)
       if (valid_row) p.lse[(int64_t)head * p.total_q + qrow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sh.o_free);
+      if (lane == 0) {
+        ptx::mbar_arrive(&sh.o_free[tile]);
+        ptx::mbar_arrive(&sh.unit_empty[slot]);
+      }
+      ++ucnt;
     }
   }
 
   // ------------------------------------------------------------------------------------ teardown
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -196,7 +196,7 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
   const int B = dims->num_seqs, H = dims->num_kv_heads, P = dims->page_size;
   if (B > 0 && (!ctx_len || !q_len || !cls || !page_table_offs)) return SEGPAGED_ERR_NULL;
   const int G = dims->num_q_heads / H;
-  const int npos = 128 / G;
+  const int npos = 2 * (128 / G);   // a unit is two 128-row query tiles sharing their K/V tiles
   const int ppt = 128 / P;
   std::vector<segpaged_unit> out;
   int32_t qrow = 0;

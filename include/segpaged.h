@@ -132,7 +132,7 @@ int segpaged_build(const segpaged_dims* dims, const void* k_dense, const void* v
 
 /*
  * SELECTVISIBLESTATE: plan the prefill work (host only).
- * Splits every (sequence, KV head) into query tiles of 128/G positions x G query heads, records for
+ * Splits every (sequence, KV head) into units of 2 x 128/G positions x G query heads, records for
  * each tile the page ranges its queries can see (the sink pages and the window pages, in page-table
  * index space) and sorts the units by their number of 128-key tiles, longest first.
  *   ctx_len, q_len (host) [B]; cls (host) [B*Hkv]; page_table_offs (host) [B*Hkv+1] (the same

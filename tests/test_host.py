@@ -100,7 +100,7 @@ def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes):
         covered = set()
         for lp in lps:
             covered.update(range(lp * P, lp * P + P))
-        assert 1 <= u[U_NPOS] <= 128 // G
+        assert 1 <= u[U_NPOS] <= 256 // G
         for r in range(int(u[U_NPOS])):
             i = int(u[U_POS0]) + r
             row = int(u[U_QROW]) + r
