@@ -347,8 +347,21 @@ def run_ours(args, rank, world, local):
     value = world * flops_step * args.steps / (ms_total * 1e-3) / 1e12
     achieved = sum(flops_layer[li] * len(prefill_ms[li]) for li in prefill_ms) / (prefill_total_ms * 1e-3) / 1e12
     peaks, src = load_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    peak_bw = float(peaks.get("hbm_gbs"))
     traffic = traffic_per_launch(w.name)
+    # algorithmic bytes of each prefill launch: stored K/V pages read once, Q read, O and LSE written
+    qo_bytes = w.total_q * w.num_q_heads * (w.head_dim * 2 * 2 + 4)
+    bytes_layer = {li: runner.state[li].stored_bytes + qo_bytes for li in runner.layers}
+    t_tensor = sum(flops_layer.values()) / (peak_tf * 1e12)
+    t_hbm = sum(bytes_layer.values()) / (peak_bw * 1e9)
+    if t_hbm > t_tensor:
+        bound, unit, peak = "hbm", "GB/s", peak_bw
+        achieved = sum(bytes_layer[li] * len(prefill_ms[li]) for li in prefill_ms) / (prefill_total_ms * 1e-3) / 1e9
+        peak_name = "hbm_gbs"
+    else:
+        bound, unit, peak = "tensor", "TFLOP/s", peak_tf
+        peak_name = "bf16_tflops_sustained"
     kinds = {}
     for li in runner.layers:
         kinds.setdefault("all-global" if runner.state[li].cls[..., 0].all() else "mixed", []).append(li)
@@ -383,9 +396,12 @@ def run_ours(args, rank, world, local):
         "ms_per_layer": prefill_total_ms / args.steps / n_layers,
         "prefill_ms_by_layer_kind": per_kind,
         "kv_bytes": {"segpaged": stored, "dense": dense, "ratio": dense / max(stored, 1)},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{src} bf16_tflops_sustained", "kernel": "segpaged_prefill_kernel"},
+                     "algorithmic_bytes_per_step": sum(bytes_layer.values()),
+                     "prefill_tflops": sum(flops_layer[li] * len(prefill_ms[li]) for li in prefill_ms)
+                     / (prefill_total_ms * 1e-3) / 1e12,
+                     "peak_source": f"{src} {peak_name}", "kernel": "segpaged_prefill_kernel"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps * n_layers * 2,

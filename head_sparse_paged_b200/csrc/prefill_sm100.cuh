@@ -402,10 +402,13 @@ __global__ void __launch_bounds__(384, 1)
         if (!wwait(&sh.s_full[tile], scount & 1)) { ok = false; break; }
         ++scount;
         ptx::tc_fence_after();
+        // S row in two halves: the second half's TMEM load overlaps the first half's masking and max.
         float s[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(sbuf + c * 32, reinterpret_cast<uint32_t*>(s) + c * 32);
+        ptx::tmem_ld32(sbuf, reinterpret_cast<uint32_t*>(s));
+        ptx::tmem_ld32(sbuf + 32, reinterpret_cast<uint32_t*>(s) + 32);
         ptx::tmem_ld_wait();
+        ptx::tmem_ld32(sbuf + 64, reinterpret_cast<uint32_t*>(s) + 64);
+        ptx::tmem_ld32(sbuf + 96, reinterpret_cast<uint32_t*>(s) + 96);
 
         // Logical page of every slot of this KV tile; a row needs per-column bounds only if some key
         // of the tile is invisible to it (causal edge, window edge, sink tail, or a short last tile).
@@ -424,22 +427,39 @@ __global__ void __launch_bounds__(384, 1)
             need_mask = true;
           }
         }
-        if (need_mask) {
+        // Row max as eight independent 3-input max chains per half, so no long dependency chain.
+        float mh[8];
 #pragma unroll
-          for (int c = 0; c < C::PPT; ++c) {
-            const int32_t base = lp[c] * P;
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1) ptx::tmem_ld_wait();
+          if (need_mask) {
 #pragma unroll
-            for (int r = 0; r < P; ++r) {
-              const int32_t jj = base + r;
-              const bool vis = lp[c] >= 0 && jj <= i_pos && (is_global || jj < S || jj > i_pos - W);
-              if (!vis) s[c * P + r] = -INFINITY;
+            for (int c = 0; c < C::PPT; ++c) {
+              const int32_t base = lp[c] * P;
+#pragma unroll
+              for (int r = 0; r < P; ++r) {
+                const int col = c * P + r;               // compile-time: columns outside this half skip
+                if (col < h * 64 || col >= h * 64 + 64) continue;
+                const int32_t jj = base + r;
+                const bool vis = lp[c] >= 0 && jj <= i_pos && (is_global || jj < S || jj > i_pos - W);
+                if (!vis) s[col] = -INFINITY;
+              }
             }
           }
-        }
-        float mx = fmax3(s[0], s[1], s[2]);
 #pragma unroll
-        for (int c = 3; c < 127; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
-        mx = fmaxf(mx, s[127]);
+          for (int k = 0; k < 4; ++k) {
+            const int b = h * 64 + k * 16;
+            float a = fmax3(s[b], s[b + 1], s[b + 2]);
+            a = fmax3(a, s[b + 3], s[b + 4]);
+            a = fmax3(a, s[b + 5], s[b + 6]);
+            a = fmax3(a, s[b + 7], s[b + 8]);
+            a = fmax3(a, s[b + 9], s[b + 10]);
+            a = fmax3(a, s[b + 11], s[b + 12]);
+            a = fmax3(a, s[b + 13], s[b + 14]);
+            mh[h * 4 + k] = fmaxf(a, s[b + 15]);
+          }
+        }
+        const float mx = fmaxf(fmax3(mh[0], mh[1], mh[2]), fmax3(fmax3(mh[3], mh[4], mh[5]), mh[6], mh[7]));
         const float m_tile = mx * sl2;
         const float m_new = fmaxf(m_run, m_tile);
         bool resc = false;
@@ -455,7 +475,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         const float mu = (m_run == -INFINITY) ? 0.f : m_run;
         const uint64_t nmu2 = f2_pack(-mu, -mu);
-        uint64_t sum2 = f2_pack(0.f, 0.f);
+        uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {          // two halves of 64 columns -> 32 packed P columns each
           uint32_t pk[32];
@@ -471,7 +491,7 @@ __global__ void __launch_bounds__(384, 1)
               f2_unpack(x2, x0, x1);
               p2 = f2_pack(ptx::ex2(x0), ptx::ex2(x1));
             }
-            sum2 = f2_add(sum2, p2);
+            sum2[c & 3] = f2_add(sum2[c & 3], p2);
             float p0, p1;
             f2_unpack(p2, p0, p1);
             pk[c] = ptx::pack_bf16x2(p0, p1);
@@ -498,7 +518,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         float sa, sb;
-        f2_unpack(sum2, sa, sb);
+        f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
         l_run += sa + sb;
         ptx::tmem_st_wait();
         ptx::tc_fence_before();

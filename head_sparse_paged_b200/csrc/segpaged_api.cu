@@ -258,9 +258,17 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
     }
     qrow += Lq;
   }
-  // Longest first, so the persistent grid finishes together; ties keep plan order.
+  // Longest first, so the persistent grid finishes together -- but by cost bucket (16 levels relative to
+  // the longest unit), keeping the plan order (sequence, KV head, query tile) inside a bucket. CTAs that
+  // start together then mostly work on the same head and sweep its pages in step, so a page is fetched
+  // from HBM once and served from L2 to the other CTAs, instead of every CTA streaming a different head.
+  int32_t max_cost = 1;
+  for (const auto& u : out) max_cost = std::max(max_cost, u.v[U_NTILES]);
+  auto bucket = [max_cost](const segpaged_unit& u) {
+    return (int32_t)(((int64_t)u.v[U_NTILES] * 16 + max_cost / 2) / max_cost);
+  };
   std::stable_sort(out.begin(), out.end(),
-                   [](const segpaged_unit& a, const segpaged_unit& b) { return a.v[U_NTILES] > b.v[U_NTILES]; });
+                   [&](const segpaged_unit& a, const segpaged_unit& b) { return bucket(a) > bucket(b); });
   const int64_t n = (int64_t)out.size();
   if (!units) return n;
   if (capacity < n) return SEGPAGED_ERR_CAPACITY;

@@ -118,6 +118,16 @@ def qwen3_32b(globals_: int = 1) -> Workload:
                     description="Qwen3-32B-shaped layer: L=131072, Lq=8192, Hq=64, Hkv=8, D=128, P=128")
 
 
+def qwen3_32b_small_q(lq: int) -> Workload:
+    """Decode-like probe on the Qwen3-32B-shaped layer: the same L=131072 pool and class map, only the last
+    `lq` positions queried (Lq in {16, 64}), so the KV pages dominate the bytes moved."""
+    w = qwen3_32b()
+    w.name = f"qwen3-32b-lq{lq}"
+    w.q_lens = [lq]
+    w.description = f"Qwen3-32B-shaped decode-like probe: L=131072, Lq={lq}, Hq=64, Hkv=8, D=128, P=128"
+    return w
+
+
 def dsv4_flash(layers: int = 43) -> Workload:
     """DeepSeek-V4-Flash-style head split: `layers` layers of 64 MHA heads (own KV each), D=128, one sequence
     L=131072 with Lq=4096, P=128, fully shuffled pool. Layers 0-2 and the last three are all global;
@@ -150,6 +160,8 @@ WORKLOADS = {
     "llama-3.3-70b": llama_70b,
     "qwen3-32b": qwen3_32b,
     "dsv4-flash": dsv4_flash,
+    "qwen3-32b-lq16": lambda: qwen3_32b_small_q(16),
+    "qwen3-32b-lq64": lambda: qwen3_32b_small_q(64),
 }
 
 

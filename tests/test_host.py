@@ -83,9 +83,11 @@ def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes):
     seen = np.zeros((int(cu_q[-1]), Hkv), np.int32)
     ppt = 128 // P
     prev = 1 << 30
+    max_cost = max([int(u[U_NTILES]) for u in units] + [1])
     for u in units:
-        assert u[U_NTILES] <= prev  # longest first
-        prev = u[U_NTILES]
+        bucket = (int(u[U_NTILES]) * 16 + max_cost // 2) // max_cost
+        assert bucket <= prev  # longest first, by cost bucket
+        prev = bucket
         b, kh = int(u[U_SEQ]), int(u[U_KVH])
         L, Lq = ctx[b], ql[b]
         g, S, W = (int(x) for x in cls[b, kh])
