@@ -51,25 +51,34 @@ SP_HD Split storage_split(int32_t L, int32_t Lq, int32_t is_global, int32_t sink
 // of the group: two 128-row tensor-core tiles that share every K/V tile. Its keys are the pages at list
 // positions [0, a_n + b_n): list position x < a_n is table index x (sink part), list position
 // x >= a_n is table index b0 + (x - a_n) (window part). KV tiles are groups of 128/P consecutive
-// list positions; n_tiles = ceil((a_n + b_n) / (128/P)).
+// list positions, n_kv = ceil((a_n + b_n) / (128/P)) of them. A record runs KV tiles [t0, t0 + n_tiles):
+// all of them, or one chunk when a long unit is split across CTAs; a chunk writes a partial result
+// (O / l in fp32 and its LSE) into partial slot `part`, and a combine record later merges the chunks of a
+// unit in chunk order. With at most 128/G valid positions the second query tile has no rows (`half`).
 enum UnitField {
-  U_QROW = 0,   // row of the first position in Q / O (index into the packed query rows)
-  U_POS0 = 1,   // absolute position of the first row
-  U_NPOS = 2,   // valid positions in this unit (<= 2 x 128/G)
-  U_KVH = 3,    // KV head
-  U_TOFF = 4,   // offset of the head's page table
-  U_NSINK = 5,  // Split::n_sink
-  U_W0 = 6,     // Split::w0
+  U_QROW = 0,     // row of the first position in Q / O (index into the packed query rows)
+  U_POS0 = 1,     // absolute position of the first row
+  U_NPOS = 2,     // valid positions in this unit (<= 2 x 128/G)
+  U_KVH = 3,      // KV head
+  U_TOFF = 4,     // offset of the head's page table
+  U_NSINK = 5,    // Split::n_sink
+  U_W0 = 6,       // Split::w0
   U_GLOBAL = 7,
   U_SINK = 8,
   U_WIN = 9,
   U_AN = 10,
   U_B0 = 11,
   U_BN = 12,
-  U_NTILES = 13,  // < 0 marks the end of the schedule inside the kernel
+  U_NTILES = 13,  // KV tiles this record runs; < 0 marks the end of the schedule inside the kernel
   U_TOTAL = 14,   // Split::total (table length)
   U_SEQ = 15,
-  U_NFIELDS = 16
+  U_T0 = 16,      // first KV tile of this record
+  U_PART = 17,    // partial slot written by a chunk of a split unit, -1 when the record writes O directly
+  U_HALF = 18,    // 1 when the second query tile has no valid rows
+  U_NSPLIT = 19,  // chunks of the unit (combine records)
+  U_NFIELDS = 32
 };
+// A combine record reuses U_QROW, U_NPOS, U_KVH, U_SEQ, U_HALF; U_PART is its first partial slot and
+// U_NSPLIT the number of consecutive slots to merge.
 
 }  // namespace segpaged

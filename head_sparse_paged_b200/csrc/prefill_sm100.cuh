@@ -71,6 +71,8 @@ struct PrefillParams {
   int32_t* status;       // nullable
   __nv_bfloat16* o;      // [total_q, Hq, D]
   float* lse;            // [Hq, total_q]
+  float* part_o;         // [partial slots][256 rows][D] fp32: O / l of one chunk of a split unit
+  float* part_lse;       // [partial slots][256 rows] fp32: LSE of that chunk (natural log)
   int32_t total_q, num_q_heads, num_pages, log2_group;
   float scale_log2;      // softmax_scale * log2(e)
 };
@@ -230,18 +232,19 @@ __global__ void __launch_bounds__(384, 1)
         if (done) break;
         // both query tiles: the unit's positions [0, npos) and [npos, 2 npos)
         if (!ptx::mbar_wait(&sh.q_empty, (ring & 1) ^ 1, abort, status, kStatusTimeout)) break;
-        ptx::mbar_arrive_expect_tx(&sh.q_full, 2 * C::Q_BYTES);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
+        const int nq = U[U_HALF] ? 1 : 2;   // a half unit has no rows in its second query tile
+        ptx::mbar_arrive_expect_tx(&sh.q_full, nq * C::Q_BYTES);
+        for (int t = 0; t < nq; ++t)
 #pragma unroll
           for (int h = 0; h < C::NH; ++h)
             ptx::tma_load_3d(sQ + t * C::Q_BYTES + h * C::BLK, &tm_q, h * 64, U[U_KVH] * G, U[U_QROW] + t * npos,
                              &sh.q_full);
         const int32_t npages = U[U_AN] + U[U_BN];
+        const int32_t t0 = U[U_T0];
         const int32_t ntiles = U[U_NTILES];
         const int64_t toff = U[U_TOFF];
         bool ok = true;
-        for (int32_t j = 0; j < ntiles && ok; ++j) {
+        for (int32_t j = t0; j < t0 + ntiles && ok; ++j) {
           int32_t pages[C::PPT];
           int32_t n_ok = 0;
 #pragma unroll
@@ -289,13 +292,13 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 9 && lane == 0) {
       // -------------------------------------------------------------------------- MMA issuer
       const uint32_t q_base = ptx::smem_addr(sQ), kv_base = ptx::smem_addr(sKV);
-      uint32_t kv_item = 0, ucnt = 0, pcount[2] = {0, 0};
+      uint32_t kv_item = 0, act[2] = {0, 0}, pcount[2] = {0, 0};
       bool ok = true;
       // O_t (+)= P_t V for the V tile in KV item vi; `first` starts the unit's accumulation.
       auto issue_pv = [&](int t, uint32_t vi, bool first) -> bool {
         if (!ptx::mbar_wait(&sh.p_full[t], pcount[t] & 1, abort, status, kStatusTimeout)) return false;
         ++pcount[t];
-        if (first && ucnt > 0 && !ptx::mbar_wait(&sh.o_free[t], (ucnt - 1) & 1, abort, status, kStatusTimeout))
+        if (first && act[t] > 0 && !ptx::mbar_wait(&sh.o_free[t], (act[t] - 1) & 1, abort, status, kStatusTimeout))
           return false;
         const int s = vi % C::NSLOT;
         if (t == 0 && !ptx::mbar_wait(&sh.kv_full[s], (vi / C::NSLOT) & 1, abort, status, kStatusTimeout))
@@ -325,9 +328,10 @@ __global__ void __launch_bounds__(384, 1)
         const int slot = ring & 1;
         if (!ptx::mbar_wait(&sh.unit_full[slot], (ring >> 1) & 1, abort, status, kStatusTimeout)) { ok = false; break; }
         const int32_t ntiles = sh.unit[slot][U_NTILES];
+        const bool two = sh.unit[slot][U_HALF] == 0;   // second query tile active
         ptx::mbar_arrive(&sh.unit_empty[slot]);
         if (ntiles < 0) break;
-        if (!ptx::mbar_wait(&sh.q_full, ucnt & 1, abort, status, kStatusTimeout)) { ok = false; break; }
+        if (!ptx::mbar_wait(&sh.q_full, (ring & 1), abort, status, kStatusTimeout)) { ok = false; break; }
         uint32_t prev_vi = 0;
         for (int32_t j = 0; j < ntiles && ok; ++j) {
           const uint32_t ki = kv_item, vi = kv_item + 1;
@@ -339,10 +343,10 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t kb = kv_base + s * C::TILE_BYTES;
           issue_s(0, kb);
           if (j > 0) {
-            if (!issue_pv(1, prev_vi, j == 1)) { ok = false; break; }
+            if (two && !issue_pv(1, prev_vi, j == 1)) { ok = false; break; }
             ptx::umma_commit(&sh.kv_empty[prev_vi % C::NSLOT]);
           }
-          issue_s(1, kb);
+          if (two) issue_s(1, kb);
           ptx::umma_commit(&sh.kv_empty[s]);
           if (j == ntiles - 1) ptx::umma_commit(&sh.q_empty);
           prev_vi = vi;
@@ -351,10 +355,13 @@ __global__ void __launch_bounds__(384, 1)
         // the unit's last PV of each tile publishes its O
         if (!issue_pv(0, prev_vi, ntiles == 1)) break;
         ptx::umma_commit(&sh.o_full[0]);
-        if (!issue_pv(1, prev_vi, ntiles == 1)) break;
-        ptx::umma_commit(&sh.o_full[1]);
+        if (two) {
+          if (!issue_pv(1, prev_vi, ntiles == 1)) break;
+          ptx::umma_commit(&sh.o_full[1]);
+        }
         ptx::umma_commit(&sh.kv_empty[prev_vi % C::NSLOT]);
-        ++ucnt;
+        ++act[0];
+        if (two) ++act[1];
       }
       // Drain: every MMA this CTA issued has completed before tensor memory is released.
       ptx::umma_commit(&sh.mma_drain);
@@ -383,11 +390,13 @@ __global__ void __launch_bounds__(384, 1)
       // the epilogue, and the producer refills a slot only once every consumer has released it.
       const int32_t* u = sh.unit[slot];
       const int32_t ntiles = u[U_NTILES];
-      if (ntiles < 0) {
+      if (ntiles < 0 || (tile == 1 && u[U_HALF])) {   // end of schedule, or no rows for this tile
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
-        break;
+        if (ntiles < 0) break;
+        continue;
       }
+      const int32_t t0 = u[U_T0];
       const int32_t pslot = tile * npos + (row >> p.log2_group);
       const bool valid_row = pslot < u[U_NPOS];
       const int32_t i_pos = u[U_POS0] + (valid_row ? pslot : u[U_NPOS] - 1);
@@ -416,7 +425,7 @@ __global__ void __launch_bounds__(384, 1)
         bool need_mask = false;
 #pragma unroll
         for (int c = 0; c < C::PPT; ++c) {
-          const int32_t x = j * C::PPT + c;
+          const int32_t x = (t0 + j) * C::PPT + c;
           if (x < npages) {
             lp[c] = unit_logical_page(u, unit_table_index(u, x));
             const int32_t j0 = lp[c] * P, j1 = j0 + P - 1;
@@ -530,6 +539,35 @@ __global__ void __launch_bounds__(384, 1)
       // ------------------------------------------------------------------------------ epilogue
       if (!wwait(&sh.o_full[tile], ucnt & 1)) break;
       ptx::tc_fence_after();
+      const int32_t part = u[U_PART];
+      if (part >= 0) {
+        // one chunk of a split unit: O / l in fp32 and the chunk's LSE, for the combine pass; a row that
+        // saw no visible key in this chunk writes O = 0 and LSE = -inf
+        const bool empty = (m_run == -INFINITY) || !(l_run > 0.f);
+        const float inv_l = empty ? 0.f : 1.0f / l_run;
+        const int64_t prow = (int64_t)part * 256 + tile * 128 + row;
+        float* dst = p.part_o + prow * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(obuf + c * 32, r);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            reinterpret_cast<float4*>(dst + c * 32)[k] =
+                make_float4(__uint_as_float(r[4 * k]) * inv_l, __uint_as_float(r[4 * k + 1]) * inv_l,
+                            __uint_as_float(r[4 * k + 2]) * inv_l, __uint_as_float(r[4 * k + 3]) * inv_l);
+        }
+        p.part_lse[prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(&sh.o_free[tile]);
+          ptx::mbar_arrive(&sh.unit_empty[slot]);
+        }
+        ++ucnt;
+        continue;
+      }
       const float inv_l = 1.0f / l_run;
       const int64_t qrow = (int64_t)u[U_QROW] + pslot;
       __nv_bfloat16* orow = p.o + (qrow * p.num_q_heads + head) * D;

@@ -16,6 +16,7 @@
 
 #include "../../include/segpaged.h"
 #include "build_kernel.cuh"
+#include "combine_kernel.cuh"
 #include "plan.h"
 #include "prefill_sm100.cuh"
 
@@ -105,6 +106,7 @@ const char* segpaged_error_string(int code) {
     case SEGPAGED_ERR_CAPACITY: return "output array too small";
     case SEGPAGED_ERR_CUDA: return "a CUDA runtime or driver call failed";
     case SEGPAGED_ERR_ALIGN: return "a base pointer is not 16-byte aligned";
+    case SEGPAGED_ERR_UNSUPPORTED: return "the plan splits units; this entry point needs a plan made with split_ctas = 0";
     default: return "unknown error";
   }
 }
@@ -189,14 +191,15 @@ int segpaged_build(const segpaged_dims* dims, const void* k_dense, const void* v
 }
 
 int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
-                              const segpaged_head_class* cls, const int32_t* page_table_offs, segpaged_unit* units,
-                              int64_t capacity) {
+                              const segpaged_head_class* cls, const int32_t* page_table_offs, int32_t split_ctas,
+                              segpaged_unit* units, int64_t capacity, segpaged_plan_info* info) {
   int rc = check_dims(dims);
   if (rc) return rc;
   const int B = dims->num_seqs, H = dims->num_kv_heads, P = dims->page_size;
   if (B > 0 && (!ctx_len || !q_len || !cls || !page_table_offs)) return SEGPAGED_ERR_NULL;
   const int G = dims->num_q_heads / H;
-  const int npos = 2 * (128 / G);   // a unit is two 128-row query tiles sharing their K/V tiles
+  const int npos_tile = 128 / G;
+  const int npos = 2 * npos_tile;   // a unit is two 128-row query tiles sharing their K/V tiles
   const int ppt = 128 / P;
   std::vector<segpaged_unit> out;
   int32_t qrow = 0;
@@ -253,22 +256,74 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
         u.v[U_NTILES] = (int32_t)ceil_div(a_n + b_n, ppt);
         u.v[U_TOTAL] = sp.total;
         u.v[U_SEQ] = b;
+        u.v[U_T0] = 0;
+        u.v[U_PART] = -1;
+        u.v[U_HALF] = nv <= npos_tile ? 1 : 0;
+        u.v[U_NSPLIT] = 0;
         out.push_back(u);
       }
     }
     qrow += Lq;
   }
+  // Tensor work of a record: KV tiles x query tiles it runs.
+  auto cost = [](const segpaged_unit& u) { return (int64_t)u.v[U_NTILES] * (u.v[U_HALF] ? 1 : 2); };
+  // Split long units across CTAs when one unit alone would exceed a CTA's fair share of the work (short
+  // query ranges, decode-like tiles): chunks of at least 8 KV tiles, sized for about two chunks per CTA.
+  std::vector<segpaged_unit> groups;
+  int32_t slots = 0;
+  if (split_ctas > 0 && !out.empty()) {
+    int64_t total = 0, longest = 0;
+    for (const auto& u : out) {
+      total += cost(u);
+      longest = std::max(longest, cost(u));
+    }
+    if (longest * split_ctas > total) {
+      const int64_t target = ceil_div(total, 2 * (int64_t)split_ctas);
+      std::vector<segpaged_unit> work;
+      for (const auto& u : out) {
+        const int32_t weight = u.v[U_HALF] ? 1 : 2;
+        const int32_t n = u.v[U_NTILES];
+        int32_t chunk = (int32_t)std::max<int64_t>(8, ceil_div(target, weight));
+        chunk = std::max<int32_t>(chunk, (int32_t)ceil_div(n, kCombineMaxSplit));   // at most 256 chunks
+        if (n <= chunk) {
+          work.push_back(u);
+          continue;
+        }
+        const int32_t k = (int32_t)ceil_div(n, chunk);
+        segpaged_unit g = u;
+        g.v[U_PART] = slots;
+        g.v[U_NSPLIT] = k;
+        g.v[U_NTILES] = 0;
+        groups.push_back(g);
+        int32_t t0 = 0;
+        for (int32_t c = 0; c < k; ++c) {
+          const int32_t len = n / k + (c < n % k ? 1 : 0);
+          segpaged_unit w = u;
+          w.v[U_T0] = t0;
+          w.v[U_NTILES] = len;
+          w.v[U_PART] = slots++;
+          work.push_back(w);
+          t0 += len;
+        }
+      }
+      out.swap(work);
+    }
+  }
   // Longest first, so the persistent grid finishes together -- but by cost bucket (16 levels relative to
-  // the longest unit), keeping the plan order (sequence, KV head, query tile) inside a bucket. CTAs that
-  // start together then mostly work on the same head and sweep its pages in step, so a page is fetched
-  // from HBM once and served from L2 to the other CTAs, instead of every CTA streaming a different head.
-  int32_t max_cost = 1;
-  for (const auto& u : out) max_cost = std::max(max_cost, u.v[U_NTILES]);
-  auto bucket = [max_cost](const segpaged_unit& u) {
-    return (int32_t)(((int64_t)u.v[U_NTILES] * 16 + max_cost / 2) / max_cost);
-  };
+  // the longest record), keeping the plan order (sequence, KV head, query tile, chunk) inside a bucket.
+  // CTAs that start together then mostly work on the same head and sweep its pages in step, so a page is
+  // fetched from HBM once and served from L2 to the other CTAs, instead of every CTA streaming another head.
+  int64_t max_cost = 1;
+  for (const auto& u : out) max_cost = std::max(max_cost, cost(u));
+  auto bucket = [&](const segpaged_unit& u) { return (cost(u) * 16 + max_cost / 2) / max_cost; };
   std::stable_sort(out.begin(), out.end(),
                    [&](const segpaged_unit& a, const segpaged_unit& b) { return bucket(a) > bucket(b); });
+  if (info) {
+    info->num_units = (int64_t)out.size();
+    info->num_groups = (int64_t)groups.size();
+    info->num_partials = slots;
+  }
+  out.insert(out.end(), groups.begin(), groups.end());
   const int64_t n = (int64_t)out.size();
   if (!units) return n;
   if (capacity < n) return SEGPAGED_ERR_CAPACITY;
@@ -276,9 +331,16 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
   return n;
 }
 
-size_t segpaged_prefill_workspace_bytes(int64_t num_units) {
-  (void)num_units;
-  return 256;
+namespace {
+constexpr size_t kCounterBytes = 256;
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t partial_o_bytes(int64_t slots, int D) { return align256((size_t)slots * 256 * D * sizeof(float)); }
+}  // namespace
+
+size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpaged_plan_info* info) {
+  if (!dims || !info || info->num_partials < 0) return kCounterBytes;
+  return kCounterBytes + partial_o_bytes(info->num_partials, dims->head_dim) +
+         align256((size_t)info->num_partials * 256 * sizeof(float));
 }
 
 }  // extern "C"
@@ -304,18 +366,30 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 
 }  // namespace
 
+template <int D>
+int launch_combine(const CombineParams& c, cudaStream_t st) {
+  if (c.num_groups <= 0) return SEGPAGED_OK;
+  const dim3 grid((unsigned)std::min<int64_t>(c.num_groups, 65535), 128);   // records x row pairs
+  segpaged_combine_kernel<D><<<grid, 256, 0, st>>>(c);
+  return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
+}
+
 extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
                                      const void* v_pool, const int32_t* page_table, int64_t page_table_len,
-                                     const segpaged_unit* units, int64_t num_units, float softmax_scale, void* o,
-                                     float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                                     const segpaged_unit* plan, const segpaged_plan_info* info, float softmax_scale,
+                                     void* o, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
                                      void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
-  if (num_units < 0 || total_q < 0 || page_table_len < 0 || num_units > INT32_MAX) return SEGPAGED_ERR_DIMS;
+  if (!info) return SEGPAGED_ERR_NULL;
+  const int64_t num_units = info->num_units;
+  if (num_units < 0 || info->num_groups < 0 || info->num_partials < 0 || total_q < 0 || page_table_len < 0 ||
+      num_units > INT32_MAX || info->num_groups > INT32_MAX)
+    return SEGPAGED_ERR_DIMS;
   if (num_units == 0) return SEGPAGED_OK;
-  if (!q || !k_pool || !v_pool || !page_table || !units || !o || !lse || !workspace) return SEGPAGED_ERR_NULL;
-  if (workspace_bytes < segpaged_prefill_workspace_bytes(num_units)) return SEGPAGED_ERR_CAPACITY;
-  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o) || !aligned16(units) ||
+  if (!q || !k_pool || !v_pool || !page_table || !plan || !o || !lse || !workspace) return SEGPAGED_ERR_NULL;
+  if (workspace_bytes < segpaged_prefill_workspace_bytes(dims, info)) return SEGPAGED_ERR_CAPACITY;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o) || !aligned16(plan) ||
       !aligned16(workspace))
     return SEGPAGED_ERR_ALIGN;
   if (total_q < 1 || dims->num_pages < 1) return SEGPAGED_ERR_DIMS;
@@ -332,23 +406,27 @@ extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, i
   if (sms <= 0) return SEGPAGED_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), st) != cudaSuccess) return SEGPAGED_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   PrefillParams p;
   p.page_table = page_table;
   p.page_table_len = page_table_len;
-  p.units = reinterpret_cast<const int32_t*>(units);
+  p.units = reinterpret_cast<const int32_t*>(plan);
   p.num_units = (int32_t)num_units;
-  p.counter = static_cast<int32_t*>(workspace);
+  p.counter = reinterpret_cast<int32_t*>(ws);
   p.status = status;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
+  p.part_o = reinterpret_cast<float*>(ws + kCounterBytes);
+  p.part_lse = reinterpret_cast<float*>(ws + kCounterBytes + partial_o_bytes(info->num_partials, D));
   p.total_q = total_q;
   p.num_q_heads = Hq;
   p.num_pages = dims->num_pages;
   p.log2_group = log2_int(G);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   const int grid = (int)std::min<int64_t>(num_units, sms);
+  rc = SEGPAGED_ERR_DIMS;
 #define SEGPAGED_LAUNCH(DD, PP) \
-  if (D == DD && P == PP) return launch_prefill<DD, PP>(tq, tk, tv, p, grid, st);
+  if (D == DD && P == PP) rc = launch_prefill<DD, PP>(tq, tk, tv, p, grid, st);
   SEGPAGED_LAUNCH(128, 16)
   SEGPAGED_LAUNCH(128, 32)
   SEGPAGED_LAUNCH(128, 64)
@@ -358,7 +436,18 @@ extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, i
   SEGPAGED_LAUNCH(64, 64)
   SEGPAGED_LAUNCH(64, 128)
 #undef SEGPAGED_LAUNCH
-  return SEGPAGED_ERR_DIMS;
+  if (rc != SEGPAGED_OK || info->num_groups == 0) return rc;
+  CombineParams c;
+  c.records = reinterpret_cast<const int32_t*>(plan) + num_units * U_NFIELDS;
+  c.num_groups = (int32_t)info->num_groups;
+  c.part_o = p.part_o;
+  c.part_lse = p.part_lse;
+  c.o = p.o;
+  c.lse = lse;
+  c.total_q = total_q;
+  c.num_q_heads = Hq;
+  c.log2_group = p.log2_group;
+  return D == 128 ? launch_combine<128>(c, st) : launch_combine<64>(c, st);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -372,7 +461,7 @@ extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, i
 // contents, so the counter is cleared on every call; calls whose work overlaps on the GPU race on it.
 // ------------------------------------------------------------------------------------------------
 namespace {
-constexpr int64_t kNoAllocMaxUnits = 32768;   // the most work units one call accepts
+constexpr int64_t kNoAllocMaxUnits = 16384;   // the most work units one call accepts
 constexpr int64_t kNoAllocUnitOffset = 64;    // int32 words before the unit list (counter in word 0)
 }  // namespace
 
@@ -409,6 +498,9 @@ extern "C" int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const vo
   if (num_units > kNoAllocMaxUnits) return SEGPAGED_ERR_CAPACITY;
   if (num_units == 0) return SEGPAGED_OK;
   if (!units_host) return SEGPAGED_ERR_NULL;
+  // The static array holds no partial results, so split plans (chunks or combine records) are refused.
+  for (int64_t i = 0; i < num_units; ++i)
+    if (units_host[i].v[U_PART] >= 0 || units_host[i].v[U_NSPLIT] > 0) return SEGPAGED_ERR_UNSUPPORTED;
   int32_t* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch))) return rc;
   int32_t* units_dev = scratch + kNoAllocUnitOffset;
@@ -417,7 +509,11 @@ extern "C" int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const vo
       cudaSuccess)
     return SEGPAGED_ERR_CUDA;
   // The work counter (word 0) is zeroed on the stream by segpaged_attn_prefill before its launch.
+  segpaged_plan_info info;
+  info.num_units = num_units;
+  info.num_groups = 0;
+  info.num_partials = 0;
   return segpaged_attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len,
-                               reinterpret_cast<const segpaged_unit*>(units_dev), num_units, softmax_scale, o, lse,
+                               reinterpret_cast<const segpaged_unit*>(units_dev), &info, softmax_scale, o, lse,
                                scratch, kNoAllocUnitOffset * sizeof(int32_t), status, stream);
 }

@@ -24,7 +24,8 @@ class LayerState:
     pages_per_head: np.ndarray
     table: np.ndarray          # int32, physical ids
     offs: np.ndarray           # int32 [B*Hkv+1]
-    units: np.ndarray | None = None
+    units: np.ndarray | None = None       # plan records (work units, then combine records)
+    info: dict | None = None
     table_dev: torch.Tensor | None = None
     offs_dev: torch.Tensor | None = None
     cls_dev: torch.Tensor | None = None
@@ -47,9 +48,12 @@ class Runner:
     """
 
     def __init__(self, w: synth.Workload, device="cuda", layers=None, keep_dense=False, page_seed_offset=0,
-                 shared_dense=False):
+                 shared_dense=False, split_ctas=None):
         self.w = w
         self.device = torch.device(device)
+        # long units are split across CTAs when one alone exceeds a CTA's share (short query ranges)
+        self.split_ctas = (torch.cuda.get_device_properties(self.device).multi_processor_count
+                           if split_ctas is None else int(split_ctas))
         self.layers = list(range(w.layers)) if layers is None else list(layers)
         self.keep_dense = keep_dense or shared_dense
         self.shared_dense = shared_dense
@@ -79,8 +83,7 @@ class Runner:
         self.cu_k_dev = torch.from_numpy(w.cu_k()).to(self.device)
         self.ql_dev = torch.from_numpy(self.ql).to(self.device)
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
-        self.workspace = torch.zeros(max(sp.segpaged_prefill_workspace_bytes(0) // 4, 64), dtype=torch.int32,
-                                     device=self.device)
+        self.workspace = None
         self.rope = None
         if w.rope_theta is not None:
             self.rope = torch.from_numpy(sp.segpaged_rope_cos_sin(w.rope_theta, w.rope_deltas, D)).to(self.device)
@@ -113,6 +116,9 @@ class Runner:
         self.plan_layer(li)
         st.units_dev = torch.from_numpy(np.ascontiguousarray(st.units)).to(self.device)
         st.units_host = torch.from_numpy(np.ascontiguousarray(st.units)).pin_memory()
+        need = sp.segpaged_prefill_workspace_bytes(self.dims, st.info)
+        if self.workspace is None or self.workspace.numel() * 4 < need:
+            self.workspace = torch.zeros((need + 3) // 4, dtype=torch.int32, device=self.device)
 
     def dense_of(self, li):
         if self._tmp_dense is not None:
@@ -131,7 +137,7 @@ class Runner:
     def plan_layer(self, li):
         """Host planning of one layer's work units (SELECTVISIBLESTATE)."""
         st = self.state[li]
-        st.units = sp.segpaged_prefill_plan(self.dims, self.ctx, self.ql, st.cls, st.offs)
+        st.units, st.info = sp.segpaged_prefill_plan(self.dims, self.ctx, self.ql, st.cls, st.offs, self.split_ctas)
         return st.units
 
     def upload_plan(self, li, stream=None):
@@ -153,8 +159,8 @@ class Runner:
 
     def prefill(self, li, stream=None):
         st = self.state[li]
-        sp.segpaged_attn_prefill(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, self.scale,
-                                 st.o, st.lse, self.workspace, self.status, stream)
+        sp.segpaged_attn_prefill(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info,
+                                 self.scale, st.o, st.lse, self.workspace, self.status, stream)
 
     def step(self, stream=None):
         """Prefill of every layer (pools and plans already in place)."""

@@ -15,7 +15,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsegpaged.so")
-UNIT_FIELDS = 16
+UNIT_FIELDS = 32
 
 STATUS_PAGE_ID = 1
 STATUS_TABLE = 2
@@ -32,6 +32,10 @@ class SegPagedError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: {error_string(code)} (code {code})")
         self.code = code
+
+
+class _PlanInfo(ctypes.Structure):
+    _fields_ = [("num_units", ctypes.c_int64), ("num_groups", ctypes.c_int64), ("num_partials", ctypes.c_int64)]
 
 
 class _Dims(ctypes.Structure):
@@ -66,12 +70,13 @@ def _load():
     lib.segpaged_rope_cos_sin.argtypes = [ctypes.c_double, vp, i32, i32, vp]
     lib.segpaged_build.restype = ctypes.c_int
     lib.segpaged_build.argtypes = [dp] + [vp] * 12
+    ip = ctypes.POINTER(_PlanInfo)
     lib.segpaged_prefill_plan.restype = i64
-    lib.segpaged_prefill_plan.argtypes = [dp, vp, vp, vp, vp, vp, i64]
+    lib.segpaged_prefill_plan.argtypes = [dp, vp, vp, vp, vp, i32, vp, i64, ip]
     lib.segpaged_prefill_workspace_bytes.restype = ctypes.c_size_t
-    lib.segpaged_prefill_workspace_bytes.argtypes = [i64]
+    lib.segpaged_prefill_workspace_bytes.argtypes = [dp, ip]
     lib.segpaged_attn_prefill.restype = ctypes.c_int
-    lib.segpaged_attn_prefill.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, i64, ctypes.c_float, vp, vp, vp,
+    lib.segpaged_attn_prefill.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, ip, ctypes.c_float, vp, vp, vp,
                                           ctypes.c_size_t, vp, vp]
     lib.segpaged_attn_prefill_noalloc.restype = ctypes.c_int
     lib.segpaged_attn_prefill_noalloc.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, i64, ctypes.c_float, vp, vp, vp, vp]
@@ -156,34 +161,43 @@ def segpaged_build(dims: Dims, k_dense, v_dense, cu_seqlens_k, q_len, cls, page_
         raise SegPagedError(r, "segpaged_build")
 
 
-def segpaged_prefill_plan(dims: Dims, ctx_len, q_len, cls, page_table_offs) -> np.ndarray:
-    """Work units (int32 [n, 16], longest first) for segpaged_attn_prefill. Host only."""
+def _info(d: dict) -> _PlanInfo:
+    return _PlanInfo(int(d["num_units"]), int(d["num_groups"]), int(d["num_partials"]))
+
+
+def segpaged_prefill_plan(dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas: int = 0):
+    """(records int32 [n, 32], info dict). Records [0, num_units) are work units (longest first by cost
+    bucket), the rest combine records of split units. split_ctas > 0 lets long units be split across that
+    many concurrent CTAs (the SM count); 0 never splits. Host only."""
     B, H = dims.num_seqs, dims.num_kv_heads
     L, Lq = _host_i32(ctx_len, B), _host_i32(q_len, B)
     c, offs = _host_i32(cls, B * H * 3), _host_i32(page_table_offs, B * H + 1)
     d = dims.c()
-    n = _lib.segpaged_prefill_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), None, 0)
+    info = _PlanInfo()
+    n = _lib.segpaged_prefill_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), int(split_ctas), None, 0,
+                                   ctypes.byref(info))
     if n < 0:
         raise SegPagedError(int(n), "segpaged_prefill_plan")
     units = np.zeros((max(n, 1), UNIT_FIELDS), np.int32)
-    n2 = _lib.segpaged_prefill_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), _hp(units), n)
+    n2 = _lib.segpaged_prefill_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), int(split_ctas), _hp(units), n,
+                                    ctypes.byref(info))
     if n2 < 0:
         raise SegPagedError(int(n2), "segpaged_prefill_plan")
-    return units[:n]
+    return units[:n], {"num_units": info.num_units, "num_groups": info.num_groups, "num_partials": info.num_partials}
 
 
-def segpaged_prefill_workspace_bytes(num_units: int) -> int:
-    return int(_lib.segpaged_prefill_workspace_bytes(int(num_units)))
+def segpaged_prefill_workspace_bytes(dims: Dims, info: dict) -> int:
+    return int(_lib.segpaged_prefill_workspace_bytes(ctypes.byref(dims.c()), ctypes.byref(_info(info))))
 
 
-def segpaged_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, units, softmax_scale, o, lse, workspace,
+def segpaged_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, plan, info: dict, softmax_scale, o, lse, workspace,
                           status=None, stream=None):
-    """O [total_q, Hq, D] bf16 and LSE [Hq, total_q] float32, written in place (CUDA tensors)."""
+    """O [total_q, Hq, D] bf16 and LSE [Hq, total_q] float32, written in place (CUDA tensors).
+    plan: the plan's records on the device; info: the dict segpaged_prefill_plan returned."""
     bf = torch.bfloat16
-    n_units = units.shape[0]
     r = _lib.segpaged_attn_prefill(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]), _dev(k_pool, bf, "k_pool"),
                                    _dev(v_pool, bf, "v_pool"), _dev(page_table, torch.int32, "page_table"),
-                                   int(page_table.numel()), _dev(units, torch.int32, "units"), int(n_units),
+                                   int(page_table.numel()), _dev(plan, torch.int32, "plan"), ctypes.byref(_info(info)),
                                    float(softmax_scale), _dev(o, bf, "o"), _dev(lse, torch.float32, "lse"),
                                    _dev(workspace, None, "workspace"), int(workspace.numel() * workspace.element_size()),
                                    _dev(status, torch.int32, "status"), _stream(stream))
@@ -191,14 +205,15 @@ def segpaged_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, units, soft
         raise SegPagedError(r, "segpaged_attn_prefill")
 
 
-NOALLOC_MAX_UNITS = 32768
+NOALLOC_MAX_UNITS = 16384
 
 
 def segpaged_attn_prefill_noalloc(dims: Dims, q, k_pool, v_pool, page_table, units_host, softmax_scale, o, lse,
                                   status=None, stream=None):
     """segpaged_attn_prefill for callers that cannot allocate device memory: the plan comes straight from
     the host (int32 [n, 16] from segpaged_prefill_plan) and the library's own static device array holds
-    it and the work counter. At most NOALLOC_MAX_UNITS units; calls that overlap on the GPU race."""
+    it and the work counter. At most NOALLOC_MAX_UNITS units, from a plan made with split_ctas = 0; calls
+    that overlap on the GPU race."""
     bf = torch.bfloat16
     units = np.ascontiguousarray(np.asarray(units_host, dtype=np.int32).reshape(-1, UNIT_FIELDS))
     r = _lib.segpaged_attn_prefill_noalloc(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]),

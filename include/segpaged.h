@@ -59,6 +59,7 @@ extern "C" {
 #define SEGPAGED_ERR_CAPACITY (-6)  /* output array too small */
 #define SEGPAGED_ERR_CUDA (-7)      /* a CUDA runtime/driver call failed */
 #define SEGPAGED_ERR_ALIGN (-8)     /* a base pointer is not 16-byte aligned */
+#define SEGPAGED_ERR_UNSUPPORTED (-9) /* the plan splits units, which this entry point does not accept */
 
 #define SEGPAGED_STATUS_PAGE_ID 1   /* a page id was outside [0, num_pages); it was clamped */
 #define SEGPAGED_STATUS_TABLE 2     /* a head's page-table length disagreed with the storage rule */
@@ -81,11 +82,20 @@ typedef struct {
   int32_t window;     /* W >= 1, local heads only */
 } segpaged_head_class;
 
-/* One prefill work unit: a (sequence, KV head, query tile) with its visible page ranges.
- * Produced by segpaged_prefill_plan; its fields are private to the library. 64 bytes. */
+/* One record of a prefill plan: a work unit -- a (sequence, KV head) and up to 2 x 128/G query
+ * positions, with its visible page ranges and the KV tiles it runs -- or a combine record that merges
+ * the chunks of a split unit. Produced by segpaged_prefill_plan; the fields are private. 128 bytes. */
 typedef struct {
-  int32_t v[16];
+  int32_t v[32];
 } segpaged_unit;
+
+/* Shape of a plan: records [0, num_units) are work units, records [num_units, num_units + num_groups)
+ * combine records; num_partials partial-result slots live in the workspace. */
+typedef struct {
+  int64_t num_units;
+  int64_t num_groups;
+  int64_t num_partials;
+} segpaged_plan_info;
 
 /* Text for an error code (static storage). */
 const char* segpaged_error_string(int code);
@@ -132,34 +142,42 @@ int segpaged_build(const segpaged_dims* dims, const void* k_dense, const void* v
 
 /*
  * SELECTVISIBLESTATE: plan the prefill work (host only).
- * Splits every (sequence, KV head) into units of 2 x 128/G positions x G query heads, records for
- * each tile the page ranges its queries can see (the sink pages and the window pages, in page-table
- * index space) and sorts the units by their number of 128-key tiles, longest first.
+ * Splits every (sequence, KV head) into units of 2 x 128/G positions x G query heads (two 128-row
+ * tensor-core tiles sharing each K/V tile), records for each the page ranges its queries can see (the
+ * sink pages and the window pages, in page-table index space) and orders them longest-first by cost
+ * bucket, keeping units of one head together inside a bucket.
+ * With split_ctas > 0 (the number of CTAs that run concurrently, e.g. the SM count) and a unit longer
+ * than a CTA's fair share of the work -- short query ranges, decode-like tiles -- long units are cut
+ * into chunks of at least 8 KV tiles; each chunk writes a partial result and a combine record merges
+ * them in chunk order (deterministic). split_ctas = 0 never splits.
  *   ctx_len, q_len (host) [B]; cls (host) [B*Hkv]; page_table_offs (host) [B*Hkv+1] (the same
  *   offsets later given to the device), checked against the storage rule.
- *   units (host, nullable) [capacity].
- * Returns the number of units (also when units is NULL, to size the array), or an error code.
- * The caller copies the units to device memory for segpaged_attn_prefill; a plan stays valid for
- * any call with the same lengths, classes and offsets (e.g. every layer sharing a class map).
+ *   units (host, nullable) [capacity]; info (host, nullable) receives the plan's shape.
+ * Returns the number of records (work units + combine records; also when units is NULL, to size the
+ * array), or an error code. The caller copies the records to device memory for segpaged_attn_prefill;
+ * a plan stays valid for any call with the same lengths, classes and offsets.
  * Source: the SELECTVISIBLESTATE adapter, which picks the local-head KV to reuse and the global-head
  *   ranges to compute (aiboss88.com, 使い方, third item).
  */
 int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
-                              const segpaged_head_class* cls, const int32_t* page_table_offs,
-                              segpaged_unit* units, int64_t capacity);
+                              const segpaged_head_class* cls, const int32_t* page_table_offs, int32_t split_ctas,
+                              segpaged_unit* units, int64_t capacity, segpaged_plan_info* info);
 
-/* Device scratch bytes segpaged_attn_prefill needs (the work-unit counter). */
-size_t segpaged_prefill_workspace_bytes(int64_t num_units);
+/* Device scratch bytes segpaged_attn_prefill needs for a plan: the work counter and, for split plans,
+ * the partial results (256 x D + 256 floats per partial slot). */
+size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpaged_plan_info* info);
 
 /*
  * EXECUTE: causal attention of every query head over its own ragged paged KV (one persistent
- * kernel launch, preceded by a 4-byte memset of the workspace).
+ * kernel launch, preceded by a 4-byte memset of the workspace; for split plans followed by one
+ * combine launch).
  *   q (dev) [total_q, Hq, D] bf16.  k_pool, v_pool (dev) [num_pages, P, D] bf16.
- *   page_table (dev, int32) [page_table_len].  units (dev) [num_units] from segpaged_prefill_plan.
+ *   page_table (dev, int32) [page_table_len].
+ *   plan (dev) [info->num_units + info->num_groups] records from segpaged_prefill_plan; info (host).
  *   softmax_scale: logits are scale * q.k (1/sqrt(D) in the usual case).
  *   o (dev) [total_q, Hq, D] bf16: O = softmax(logits over the visible keys) . V.
  *   lse (dev) [Hq, total_q] float: natural-log sum of exp(logits) over the visible keys.
- *   workspace (dev) >= segpaged_prefill_workspace_bytes(num_units), 16-byte aligned.
+ *   workspace (dev) >= segpaged_prefill_workspace_bytes(dims, info), 16-byte aligned.
  *   status (dev, nullable): see SEGPAGED_STATUS_*.
  * Every stored page slot must hold finite values (segpaged_build writes zeros past the context end).
  * Sources: one fused variable-length attention kernel that keeps every head on the fast path and
@@ -169,7 +187,7 @@ size_t segpaged_prefill_workspace_bytes(int64_t num_units);
  */
 int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q,
                           const void* k_pool, const void* v_pool, const int32_t* page_table,
-                          int64_t page_table_len, const segpaged_unit* units, int64_t num_units,
+                          int64_t page_table_len, const segpaged_unit* plan, const segpaged_plan_info* info,
                           float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
                           int32_t* status, void* stream);
 
@@ -179,12 +197,13 @@ int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t tota
  * example code inside a framework's own memory pool, or a runtime that forbids allocation on its
  * request path), so they cannot provide the unit list and workspace segpaged_attn_prefill needs.
  * It computes the same result from the same arguments, except:
- *   units_host (host) [num_units] straight from segpaged_prefill_plan; it is copied on `stream` into a
+ *   units_host (host) [num_units] straight from segpaged_prefill_plan called with split_ctas = 0 (a
+ *     plan with split units returns SEGPAGED_ERR_UNSUPPORTED); it is copied on `stream` into a
  *     library-owned device array, so keep it unchanged until the stream has passed this call
  *     (a pageable buffer is staged before the call returns);
  *   no workspace arguments.
  * The library-owned array is a static device array of 2 MiB that every GPU loading the library keeps
- * until the process exits; it holds at most 32768 units (more return SEGPAGED_ERR_CAPACITY). The
+ * until the process exits; it holds at most 16384 units (more return SEGPAGED_ERR_CAPACITY). The
  * first call on a device looks up the array's device address; make that first call before any
  * stream capture. Every call on a device shares the array and it keeps the last call's contents (the
  * work counter is cleared on every call): calls whose work overlaps on the GPU race, so serialise

@@ -29,7 +29,8 @@ def lib():
 
 
 def _run(w, **kw):
-    r = Runner(w, keep_dense=True, **kw)
+    kw.setdefault("keep_dense", True)
+    r = Runner(w, **kw)
     r.step()
     torch.cuda.synchronize()
     r.check_status()
@@ -56,6 +57,51 @@ SMALL = {
     "g2-p64": lambda: synth.custom("g2-p64", [(4100, 1030)], 4, 2, 128, 64, [[(0, 70, 1024), (1, 0, 0)]], seed=25,
                                    rope_theta=1e6, rope_deltas=[1234]),
 }
+
+
+SPLIT = {
+    # decode-like query ranges over long contexts: the planner splits the long units across CTAs
+    "split-short-q": (lambda: synth.custom("split-short-q", [(3000, 7), (5000, 1), (700, 40), (2500, 130)], 8, 2, 128,
+                                           64, [[(1, 0, 0), (0, 64, 512)], [(0, 0, 300), (1, 0, 0)],
+                                                [(1, 0, 0), (1, 0, 0)], [(0, 16, 1000), (1, 0, 0)]], seed=31), None),
+    "qwen3-32b-lq16": (lambda: synth.get("qwen3-32b-lq16"), None),
+    "qwen3-32b-lq64": (lambda: synth.get("qwen3-32b-lq64"), None),
+    # splits forced on the edge shapes (every unit longer than 8 KV tiles is cut)
+    "varlen-p16-g4-forced": (lambda: synth.custom("varlen-p16-g4-forced", [(2000, 300), (37, 37), (5, 0), (900, 129)],
+                                                  8, 2, 128, 16, [[(0, 0, 100), (1, 0, 0)], [(0, 50, 3), (0, 2, 1)],
+                                                                  [(1, 0, 0), (0, 1, 1)], [(0, 17, 200), (0, 1, 31)]],
+                                                  seed=32), 1000),
+    "mha-d64-p128-forced": (SMALL["mha-d64-p128"], 1000),
+    "g2-p64-forced": (SMALL["g2-p64"], 1000),
+}
+
+
+def _every_row(name, w, r):
+    st = r.state[0]
+    k, v = r.dense[0]
+    qn, kn, vn = oracle_dense(w, st.q, k, v)
+    pb = full_problem(w, 0, qn, kn, vn)
+    items = np.array([(row, h) for row in range(w.total_q) for h in range(w.num_q_heads)], np.int64)
+    o_ref, lse_ref = lib().attention(pb, r.scale, items)
+    o = st.o.float().cpu().numpy().reshape(-1, w.head_dim)
+    lse = st.lse.cpu().numpy().T.reshape(-1)
+    compare(o, lse, o_ref, lse_ref, name)
+
+
+@pytest.mark.parametrize("name", list(SPLIT))
+def test_split_prefill_matches_oracle_every_row(name):
+    make, split = SPLIT[name]
+    w = make()
+    r = _run(w, split_ctas=split)
+    assert r.state[0].info["num_groups"] > 0, "expected a split plan"
+    _every_row(name, w, r)
+
+
+def test_split_prefill_is_bit_identical_under_page_permutation():
+    w = SPLIT["split-short-q"][0]()
+    a = _run(w)
+    b = _run(w, page_seed_offset=7)
+    assert torch.equal(a.state[0].o, b.state[0].o) and torch.equal(a.state[0].lse, b.state[0].lse)
 
 
 @pytest.mark.parametrize("name", list(SMALL))

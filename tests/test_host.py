@@ -13,8 +13,9 @@ from oracle import reference as orc
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-# Work-unit field positions (head_sparse_paged_b200/csrc/plan.h).
-U_QROW, U_POS0, U_NPOS, U_KVH, U_TOFF, U_NSINK, U_W0, U_GLOBAL, U_SINK, U_WIN, U_AN, U_B0, U_BN, U_NTILES, U_TOTAL, U_SEQ = range(16)
+# Plan record field positions (head_sparse_paged_b200/csrc/plan.h).
+(U_QROW, U_POS0, U_NPOS, U_KVH, U_TOFF, U_NSINK, U_W0, U_GLOBAL, U_SINK, U_WIN, U_AN, U_B0, U_BN, U_NTILES, U_TOTAL,
+ U_SEQ, U_T0, U_PART, U_HALF, U_NSPLIT) = range(20)
 
 
 def test_library_exports_every_declared_symbol():
@@ -69,7 +70,10 @@ EDGE = [
 ]
 
 
-def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes):
+def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes, split_ctas=0):
+    """Every (query row, head) of every sequence is run by exactly one unit, over KV tiles that together
+    hold every key the oracle says the row can see; chunks of a split unit tile its KV range exactly and
+    each combine record names its chunks' partial slots."""
     B = len(w_seqs)
     dims = sp.Dims(B, Hq, Hkv, D, P)
     ctx = [s[0] for s in w_seqs]
@@ -77,15 +81,20 @@ def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes):
     cls = np.asarray(classes, np.int32)
     _, _, per = sp.segpaged_pages_bytes(dims, ctx, ql, cls)
     offs = np.concatenate([[0], np.cumsum(per)]).astype(np.int32)
-    units = sp.segpaged_prefill_plan(dims, ctx, ql, cls, offs)
+    recs, info = sp.segpaged_prefill_plan(dims, ctx, ql, cls, offs, split_ctas)
+    nu, ng = info["num_units"], info["num_groups"]
+    assert len(recs) == nu + ng
+    units, groups = recs[:nu], recs[nu:]
     G = Hq // Hkv
     cu_q = np.concatenate([[0], np.cumsum(ql)])
     seen = np.zeros((int(cu_q[-1]), Hkv), np.int32)
     ppt = 128 // P
+    cost = [int(u[U_NTILES]) * (1 if u[U_HALF] else 2) for u in units]
+    max_cost = max(cost + [1])
     prev = 1 << 30
-    max_cost = max([int(u[U_NTILES]) for u in units] + [1])
-    for u in units:
-        bucket = (int(u[U_NTILES]) * 16 + max_cost // 2) // max_cost
+    chunks = {}
+    for u, c in zip(units, cost):
+        bucket = (c * 16 + max_cost // 2) // max_cost
         assert bucket <= prev  # longest first, by cost bucket
         prev = bucket
         b, kh = int(u[U_SEQ]), int(u[U_KVH])
@@ -94,21 +103,44 @@ def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes):
         stored = orc.stored_logical_pages(L, Lq, bool(g), S, W, P)
         assert u[U_TOTAL] == len(stored) and u[U_TOFF] == offs[b * Hkv + kh]
         npages = int(u[U_AN] + u[U_BN])
-        assert u[U_NTILES] == -(-npages // ppt)
+        n_kv = -(-npages // ppt)
+        assert 0 <= u[U_T0] and u[U_T0] + u[U_NTILES] <= n_kv and u[U_NTILES] >= 1
         idxs = [x if x < u[U_AN] else int(u[U_B0]) + x - int(u[U_AN]) for x in range(npages)]
         assert len(set(idxs)) == npages and all(0 <= x < len(stored) for x in idxs)
         lps = [x if x < u[U_NSINK] else int(u[U_W0]) + x - int(u[U_NSINK]) for x in idxs]
         assert lps == [stored[x] for x in idxs]          # table index -> logical page is the storage order
+        assert 1 <= u[U_NPOS] <= 256 // G and u[U_HALF] == (u[U_NPOS] <= 128 // G)
+        key = (b, kh, int(u[U_QROW]))
+        if u[U_PART] >= 0:
+            chunks.setdefault(key, []).append((int(u[U_T0]), int(u[U_NTILES]), int(u[U_PART])))
+            continue
+        assert u[U_T0] == 0 and u[U_NTILES] == n_kv
         covered = set()
         for lp in lps:
             covered.update(range(lp * P, lp * P + P))
-        assert 1 <= u[U_NPOS] <= 256 // G
         for r in range(int(u[U_NPOS])):
             i = int(u[U_POS0]) + r
             row = int(u[U_QROW]) + r
             assert row - cu_q[b] == i - (L - Lq)
             assert set(orc.visible_keys(bool(g), S, W, i).tolist()) <= covered
             seen[row, kh] += 1
+    slots = set()
+    for grp in groups:
+        b, kh = int(grp[U_SEQ]), int(grp[U_KVH])
+        key = (b, kh, int(grp[U_QROW]))
+        parts = sorted(chunks.pop(key))
+        assert len(parts) == grp[U_NSPLIT] >= 2
+        assert [p[2] for p in parts] == list(range(int(grp[U_PART]), int(grp[U_PART] + grp[U_NSPLIT])))
+        t = 0
+        for t0, n, _ in parts:                           # chunks tile the unit's KV range in order
+            assert t0 == t
+            t += n
+        npages = int(grp[U_AN] + grp[U_BN])
+        assert t == -(-npages // ppt)
+        slots.update(p[2] for p in parts)
+        for r in range(int(grp[U_NPOS])):
+            seen[int(grp[U_QROW]) + r, kh] += 1
+    assert not chunks and len(slots) == info["num_partials"]
     assert np.all(seen == 1)
     return units
 
@@ -116,6 +148,40 @@ def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes):
 @pytest.mark.parametrize("case", range(len(EDGE)))
 def test_plan_units_cover_every_row_once_and_every_visible_key(case):
     _units_cover_exactly(*EDGE[case])
+
+
+@pytest.mark.parametrize("case", range(len(EDGE)))
+def test_plan_with_splits_covers_every_row_once(case):
+    _units_cover_exactly(*EDGE[case], split_ctas=1000)
+
+
+def test_split_policy_on_workloads():
+    """Long-context prefill is never split; decode-like tiles and the 8K layer are."""
+    def info(w):
+        dims = sp.Dims(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.page_size)
+        _, _, per = sp.segpaged_pages_bytes(dims, w.ctx_lens, w.q_lens, w.classes[0])
+        offs = np.concatenate([[0], np.cumsum(per)]).astype(np.int32)
+        return sp.segpaged_prefill_plan(dims, w.ctx_lens, w.q_lens, w.classes[0], offs, 148)[1]
+    for name in ("qwen3-32b", "llama-3.3-70b"):
+        assert info(synth.get(name))["num_groups"] == 0, name
+    assert info(synth.dsv4_flash(layers=4))["num_groups"] == 0
+    for name in ("qwen3-32b-lq16", "qwen3-32b-lq64", "mistral-7b"):
+        i = info(synth.get(name))
+        assert i["num_groups"] > 0 and i["num_units"] >= 148, (name, i)
+
+
+def test_noalloc_refuses_split_plans():
+    """Checked on the host before any device work."""
+    w = synth.get("qwen3-32b-lq16")
+    dims = sp.Dims(1, 64, 8, 128, 128, 2000)
+    _, _, per = sp.segpaged_pages_bytes(dims, w.ctx_lens, w.q_lens, w.classes[0])
+    offs = np.concatenate([[0], np.cumsum(per)]).astype(np.int32)
+    recs, info = sp.segpaged_prefill_plan(dims, w.ctx_lens, w.q_lens, w.classes[0], offs, 148)
+    recs = np.ascontiguousarray(recs)
+    rc = sp.library().segpaged_attn_prefill_noalloc(ctypes.byref(dims.c()), None, 16, None, None, None, 0,
+                                                     recs.ctypes.data_as(ctypes.c_void_p), len(recs), 0.1, None, None,
+                                                     None, None)
+    assert rc == -9
 
 
 @pytest.mark.parametrize("name", ["tiny", "mistral-7b", "llama-3.3-70b", "qwen3-32b"])
@@ -159,7 +225,8 @@ def test_validation_errors():
     lib = sp.library()
     # NULL dims and NULL arrays
     assert lib.segpaged_pages_bytes(None, None, None, None, None, None) == -1
-    assert lib.segpaged_attn_prefill(ctypes.byref(dims.c()), None, 1, None, None, None, 0, None, 3, 1.0, None, None,
-                                     None, 256, None, None) == -1
+    info = sp._PlanInfo(3, 0, 0)
+    assert lib.segpaged_attn_prefill(ctypes.byref(dims.c()), None, 1, None, None, None, 0, None, ctypes.byref(info), 1.0,
+                                     None, None, None, 256, None, None) == -1
     assert lib.segpaged_build(ctypes.byref(dims.c()), *([None] * 12)) == -1
     assert sp.error_string(-5).startswith("page-table")
