@@ -4,10 +4,10 @@
 // chunk's softmax-weighted V sum normalised by its own row sum, and LSE_c, the natural-log sum of the
 // chunk's exponentials (-inf when the row saw no visible key in it). Exact attention over the union is
 //   LSE = log sum_c exp(LSE_c),   O = sum_c exp(LSE_c - LSE) O_c.
-// A block handles two tile rows of one combine record with four warps per row: warp part k takes the
-// chunks c = k (mod 4) (loads unrolled for memory-level parallelism) and keeps its own (max, sum, O)
-// triple; the four triples are then merged in a fixed order, so the result does not depend on which CTA
-// ran which chunk. Each lane owns D/32 columns (coalesced). HBM-bound and small.
+// One pass per row merges the chunks online (running max, rescaled sum and accumulator), four chunks'
+// loads in flight at a time; rows of records with few chunks get a warp each, rows of records with many
+// chunks a whole block whose eight per-warp results are merged in a fixed order. The order of the merge
+// depends only on the plan, never on which CTA ran which chunk. Each lane owns D/32 columns (coalesced).
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -28,14 +28,59 @@ struct CombineParams {
   int32_t total_q, num_q_heads, log2_group;
 };
 
-// grid: (combine records, 128 row pairs); block: 256 threads = 2 rows x 4 warps.
+// Online merge of chunks c = c0, c0 + stride, ... into (m, wsum, acc): loads of four chunks are issued
+// together, the running max rescales what was accumulated so far when it grows.
+template <int V>
+__device__ __forceinline__ void merge_chunks(const float* part_o, const float* part_lse, int32_t part0, int32_t nsplit,
+                                             int c0, int stride, int r, int lane, int D, float& m, float& wsum,
+                                             float (&acc)[V]) {
+  int c = c0;
+  for (; c < nsplit; c += 4 * stride) {
+    float lc[4];
+    float2 v[4][V / 2];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int cc = c + u * stride;
+      lc[u] = -INFINITY;
+      if (cc < nsplit) {
+        const int64_t slot = part0 + cc;
+        lc[u] = part_lse[slot * 256 + r];
+        const float* src = part_o + (slot * 256 + r) * D + lane * V;
+#pragma unroll
+        for (int k = 0; k < V / 2; ++k) v[u][k] = *reinterpret_cast<const float2*>(src + 2 * k);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (lc[u] == -INFINITY) continue;  // no visible key of this row in the chunk (or past the end)
+      if (lc[u] > m) {
+        const float f = (m == -INFINITY) ? 0.f : expf(m - lc[u]);
+        wsum *= f;
+#pragma unroll
+        for (int k = 0; k < V; ++k) acc[k] *= f;
+        m = lc[u];
+      }
+      const float w = expf(lc[u] - m);
+      wsum += w;
+#pragma unroll
+      for (int k = 0; k < V / 2; ++k) {
+        acc[2 * k] += w * v[u][k].x;
+        acc[2 * k + 1] += w * v[u][k].y;
+      }
+    }
+  }
+}
+
+// grid: (combine records, 256). A record with at most 16 chunks gets one warp per row (blockIdx.y picks a
+// block of 8 rows); a wider record gets all 8 warps of a block on one row (blockIdx.y is the row), warp w
+// merging chunks c = w (mod 8), and the eight partial triples are merged in order 0..7.
 template <int D>
 __global__ void __launch_bounds__(256) segpaged_combine_kernel(const CombineParams p) {
   constexpr int V = D / 32;  // columns per lane
-  __shared__ float s_m[2][4], s_sum[2][4];
-  __shared__ float s_acc[2][4][D];
+  constexpr int NW = 8;      // warps per block
+  __shared__ float s_m[NW], s_sum[NW];
+  __shared__ float s_acc[NW][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rl = warp >> 2, part = warp & 3;  // row within the block, chunk residue of this warp
   const int G = 1 << p.log2_group;
   const int npos_tile = 128 >> p.log2_group;
   for (int gi = blockIdx.x; gi < p.num_groups; gi += gridDim.x) {
@@ -43,89 +88,55 @@ __global__ void __launch_bounds__(256) segpaged_combine_kernel(const CombinePara
     const int32_t part0 = rec[U_PART], nsplit = rec[U_NSPLIT], npos = rec[U_NPOS];
     const int32_t qrow0 = rec[U_QROW], kvh = rec[U_KVH];
     const int rows = rec[U_HALF] ? 128 : 256;
-    const int r = blockIdx.y * 2 + rl;
+    const bool wide = nsplit > 16;
+    const int r = wide ? (int)blockIdx.y : (int)blockIdx.y * NW + warp;
+    if ((wide ? r : (int)blockIdx.y * NW) >= rows) continue;     // uniform for the whole block
     const int tile = r >> 7, rr = r & 127;
     const int32_t pslot = tile * npos_tile + (rr >> p.log2_group);
-    const bool active = r < rows && pslot < npos;    // uniform per row (per warp group of 4)
+    const bool active = r < rows && pslot < npos;
+    if (wide && !active) continue;                                // uniform: one row per block
     float m = -INFINITY, wsum = 0.f, acc[V];
 #pragma unroll
     for (int k = 0; k < V; ++k) acc[k] = 0.f;
-    if (active) {
-      // this warp's chunks: c = part + 4 * t, t = 0, 1, ...
-      for (int c = part + 4 * lane; c < nsplit; c += 128) m = fmaxf(m, p.part_lse[(int64_t)(part0 + c) * 256 + r]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if (m != -INFINITY) {
-        int c = part;
-        for (; c + 12 < nsplit; c += 16) {   // four chunks in flight per iteration
-          float lc[4];
-          float2 v[4][V / 2];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int64_t slot = part0 + c + 4 * u;
-            lc[u] = p.part_lse[slot * 256 + r];
-            const float* src = p.part_o + (slot * 256 + r) * D + lane * V;
-#pragma unroll
-            for (int k = 0; k < V / 2; ++k) v[u][k] = *reinterpret_cast<const float2*>(src + 2 * k);
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float w = (lc[u] == -INFINITY) ? 0.f : expf(lc[u] - m);
-            wsum += w;
-#pragma unroll
-            for (int k = 0; k < V / 2; ++k) {
-              acc[2 * k] += w * v[u][k].x;
-              acc[2 * k + 1] += w * v[u][k].y;
-            }
-          }
-        }
-        for (; c < nsplit; c += 4) {
-          const float lc = p.part_lse[(int64_t)(part0 + c) * 256 + r];
-          if (lc == -INFINITY) continue;  // no visible key of this row in the chunk
-          const float w = expf(lc - m);
-          wsum += w;
-          const float* src = p.part_o + ((int64_t)(part0 + c) * 256 + r) * D + lane * V;
-#pragma unroll
-          for (int k = 0; k < V; k += 2) {
-            const float2 vv = *reinterpret_cast<const float2*>(src + k);
-            acc[k] += w * vv.x;
-            acc[k + 1] += w * vv.y;
-          }
-        }
+    if (active) merge_chunks<V>(p.part_o, p.part_lse, part0, nsplit, wide ? warp : 0, wide ? NW : 1, r, lane, D, m,
+                                wsum, acc);
+    if (wide) {
+      if (lane == 0) {
+        s_m[warp] = m;
+        s_sum[warp] = wsum;
       }
-    }
-    if (lane == 0) {
-      s_m[rl][part] = m;
-      s_sum[rl][part] = wsum;
-    }
 #pragma unroll
-    for (int k = 0; k < V; ++k) s_acc[rl][part][lane * V + k] = acc[k];
-    __syncthreads();
-    if (active && part == 0) {
-      // merge the four warps' triples in order 0..3
-      float M = s_m[rl][0];
+      for (int k = 0; k < V; ++k) s_acc[warp][lane * V + k] = acc[k];
+      __syncthreads();
+      if (warp == 0) {
+        float M = s_m[0];
 #pragma unroll
-      for (int q = 1; q < 4; ++q) M = fmaxf(M, s_m[rl][q]);
-      float tot = 0.f, out[V];
+        for (int q = 1; q < NW; ++q) M = fmaxf(M, s_m[q]);
+        float tot = 0.f;
 #pragma unroll
-      for (int k = 0; k < V; ++k) out[k] = 0.f;
+        for (int k = 0; k < V; ++k) acc[k] = 0.f;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float f = (s_m[rl][q] == -INFINITY) ? 0.f : expf(s_m[rl][q] - M);
-        tot += f * s_sum[rl][q];
+        for (int q = 0; q < NW; ++q) {
+          const float f = (s_m[q] == -INFINITY) ? 0.f : expf(s_m[q] - M);
+          tot += f * s_sum[q];
 #pragma unroll
-        for (int k = 0; k < V; ++k) out[k] += f * s_acc[rl][q][lane * V + k];
+          for (int k = 0; k < V; ++k) acc[k] += f * s_acc[q][lane * V + k];
+        }
+        m = M;
+        wsum = tot;
       }
-      const float inv = 1.0f / tot;
+      __syncthreads();
+    }
+    if (active && (!wide || warp == 0)) {
+      const float inv = 1.0f / wsum;
       const int32_t head = kvh * G + (rr & (G - 1));
       const int64_t qrow = (int64_t)qrow0 + pslot;
       __nv_bfloat16* dst = p.o + (qrow * p.num_q_heads + head) * D + lane * V;
 #pragma unroll
       for (int k = 0; k < V; k += 2)
-        *reinterpret_cast<__nv_bfloat162*>(dst + k) = __floats2bfloat162_rn(out[k] * inv, out[k + 1] * inv);
-      if (lane == 0) p.lse[(int64_t)head * p.total_q + qrow] = M + logf(tot);
+        *reinterpret_cast<__nv_bfloat162*>(dst + k) = __floats2bfloat162_rn(acc[k] * inv, acc[k + 1] * inv);
+      if (lane == 0) p.lse[(int64_t)head * p.total_q + qrow] = m + logf(wsum);
     }
-    __syncthreads();
   }
 }
 

@@ -11,7 +11,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <queue>
 #include <vector>
 
 #include "../../include/segpaged.h"
@@ -268,7 +270,10 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
   // Tensor work of a record: KV tiles x query tiles it runs.
   auto cost = [](const segpaged_unit& u) { return (int64_t)u.v[U_NTILES] * (u.v[U_HALF] ? 1 : 2); };
   // Split long units across CTAs when one unit alone would exceed a CTA's fair share of the work (short
-  // query ranges, decode-like tiles): chunks of at least 8 KV tiles, sized for about two chunks per CTA.
+  // query ranges, decode-like tiles). A unit longer than a target T is cut into near-equal chunks of at
+  // least 4 KV tiles (at most 256 chunks). T is chosen among one to four waves of the CTAs by simulating
+  // the longest-first schedule with a fixed per-record overhead (queries, pipeline fill, partial write),
+  // so a split is only as fine as the makespan rewards; ties keep the coarser split (less partial traffic).
   std::vector<segpaged_unit> groups;
   int32_t slots = 0;
   if (split_ctas > 0 && !out.empty()) {
@@ -278,13 +283,44 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
       longest = std::max(longest, cost(u));
     }
     if (longest * split_ctas > total) {
-      const int64_t target = ceil_div(total, 2 * (int64_t)split_ctas);
+      auto chunk_of = [](const segpaged_unit& u, int64_t target) {
+        const int32_t weight = u.v[U_HALF] ? 1 : 2;
+        int32_t chunk = (int32_t)std::max<int64_t>(4, ceil_div(target, weight));
+        return std::max<int32_t>(chunk, (int32_t)ceil_div(u.v[U_NTILES], kCombineMaxSplit));
+      };
+      constexpr int64_t kRecordOverhead = 4;   // fixed cost of a record, in tile x query-tile units
+      int64_t best_target = 0, best_span = INT64_MAX;
+      for (int waves = 1; waves <= 4; ++waves) {
+        const int64_t target = ceil_div(total, (int64_t)waves * split_ctas);
+        std::vector<int64_t> items;
+        for (const auto& u : out) {
+          const int32_t n = u.v[U_NTILES], chunk = chunk_of(u, target), weight = u.v[U_HALF] ? 1 : 2;
+          if (n <= chunk) {
+            items.push_back(cost(u) + kRecordOverhead);
+            continue;
+          }
+          const int32_t k = (int32_t)ceil_div(n, chunk);
+          for (int32_t c = 0; c < k; ++c) items.push_back((int64_t)(n / k + (c < n % k ? 1 : 0)) * weight + kRecordOverhead);
+        }
+        std::sort(items.begin(), items.end(), std::greater<int64_t>());
+        std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> load;
+        for (int32_t c = 0; c < split_ctas; ++c) load.push(0);
+        int64_t span = 0;
+        for (int64_t it : items) {
+          const int64_t x = load.top() + it;
+          load.pop();
+          load.push(x);
+          span = std::max(span, x);
+        }
+        if (span < best_span) {
+          best_span = span;
+          best_target = target;
+        }
+      }
       std::vector<segpaged_unit> work;
       for (const auto& u : out) {
-        const int32_t weight = u.v[U_HALF] ? 1 : 2;
         const int32_t n = u.v[U_NTILES];
-        int32_t chunk = (int32_t)std::max<int64_t>(8, ceil_div(target, weight));
-        chunk = std::max<int32_t>(chunk, (int32_t)ceil_div(n, kCombineMaxSplit));   // at most 256 chunks
+        const int32_t chunk = chunk_of(u, best_target);
         if (n <= chunk) {
           work.push_back(u);
           continue;
@@ -369,7 +405,7 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 template <int D>
 int launch_combine(const CombineParams& c, cudaStream_t st) {
   if (c.num_groups <= 0) return SEGPAGED_OK;
-  const dim3 grid((unsigned)std::min<int64_t>(c.num_groups, 65535), 128);   // records x row pairs
+  const dim3 grid((unsigned)std::min<int64_t>(c.num_groups, 65535), 256);   // records x tile rows
   segpaged_combine_kernel<D><<<grid, 256, 0, st>>>(c);
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
 }

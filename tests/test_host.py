@@ -157,17 +157,21 @@ def test_plan_with_splits_covers_every_row_once(case):
 
 def test_split_policy_on_workloads():
     """Long-context prefill is never split; decode-like tiles and the 8K layer are."""
-    def info(w):
+    def plan(w):
         dims = sp.Dims(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.page_size)
         _, _, per = sp.segpaged_pages_bytes(dims, w.ctx_lens, w.q_lens, w.classes[0])
         offs = np.concatenate([[0], np.cumsum(per)]).astype(np.int32)
-        return sp.segpaged_prefill_plan(dims, w.ctx_lens, w.q_lens, w.classes[0], offs, 148)[1]
+        return sp.segpaged_prefill_plan(dims, w.ctx_lens, w.q_lens, w.classes[0], offs, 148)
     for name in ("qwen3-32b", "llama-3.3-70b"):
-        assert info(synth.get(name))["num_groups"] == 0, name
-    assert info(synth.dsv4_flash(layers=4))["num_groups"] == 0
+        assert plan(synth.get(name))[1]["num_groups"] == 0, name
+    assert plan(synth.dsv4_flash(layers=4))[1]["num_groups"] == 0
     for name in ("qwen3-32b-lq16", "qwen3-32b-lq64", "mistral-7b"):
-        i = info(synth.get(name))
-        assert i["num_groups"] > 0 and i["num_units"] >= 148, (name, i)
+        recs, i = plan(synth.get(name))
+        work = recs[:i["num_units"]]
+        cost = work[:, U_NTILES].astype(np.int64) * np.where(work[:, U_HALF] == 1, 1, 2)
+        share = -(-int(cost.sum()) // 148)                 # one CTA's share of the tensor work
+        assert i["num_groups"] > 0, name
+        assert cost.max() <= max(share, 16) + 2, (name, int(cost.max()), share)   # about one wave of equal pieces
 
 
 def test_noalloc_refuses_split_plans():
