@@ -211,81 +211,100 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
-    if (warp == 8 && lane == 0) {
+    if (warp == 8) {
       // ---------------------------------------------------------------------------- producer
+      // The whole warp walks the schedule; lane 0 does the barrier and TMA work, and the 32 lanes fetch
+      // the page-table entries of 32 list positions at once, so a tile's loads never wait on a lookup.
       uint32_t kv_item = 0;
       for (uint32_t ring = 0;; ++ring) {
         const int slot = ring & 1;
-        if (!ptx::mbar_wait(&sh.unit_empty[slot], ((ring >> 1) & 1) ^ 1, abort, status, kStatusTimeout)) break;
+        int go = 1;
+        if (lane == 0) go = ptx::mbar_wait(&sh.unit_empty[slot], ((ring >> 1) & 1) ^ 1, abort, status, kStatusTimeout);
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
         // claim the next unit only once a ring slot is free, so no CTA sits on work it cannot start
-        const int32_t u = atomicAdd(p.counter, 1);
+        int32_t u = 0;
+        if (lane == 0) u = atomicAdd(p.counter, 1);
+        u = __shfl_sync(0xffffffffu, u, 0);
         const bool done = u >= p.num_units;
         int32_t* U = sh.unit[slot];
         if (done) {
-          U[U_NTILES] = -1;
-        } else {
-          const int4* src = reinterpret_cast<const int4*>(p.units + (int64_t)u * U_NFIELDS);
-#pragma unroll
-          for (int i = 0; i < U_NFIELDS / 4; ++i) reinterpret_cast<int4*>(U)[i] = src[i];
+          if (lane == 0) U[U_NTILES] = -1;
+        } else if (lane < U_NFIELDS / 4) {
+          reinterpret_cast<int4*>(U)[lane] = reinterpret_cast<const int4*>(p.units + (int64_t)u * U_NFIELDS)[lane];
         }
-        ptx::mbar_arrive(&sh.unit_full[slot]);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.unit_full[slot]);
         if (done) break;
         // both query tiles: the unit's positions [0, npos) and [npos, 2 npos)
-        if (!ptx::mbar_wait(&sh.q_empty, (ring & 1) ^ 1, abort, status, kStatusTimeout)) break;
-        const int nq = U[U_HALF] ? 1 : 2;   // a half unit has no rows in its second query tile
-        ptx::mbar_arrive_expect_tx(&sh.q_full, nq * C::Q_BYTES);
-        for (int t = 0; t < nq; ++t)
+        if (lane == 0) {
+          go = ptx::mbar_wait(&sh.q_empty, (ring & 1) ^ 1, abort, status, kStatusTimeout);
+          if (go) {
+            const int nq = U[U_HALF] ? 1 : 2;   // a half unit has no rows in its second query tile
+            ptx::mbar_arrive_expect_tx(&sh.q_full, nq * C::Q_BYTES);
+            for (int t = 0; t < nq; ++t)
 #pragma unroll
-          for (int h = 0; h < C::NH; ++h)
-            ptx::tma_load_3d(sQ + t * C::Q_BYTES + h * C::BLK, &tm_q, h * 64, U[U_KVH] * G, U[U_QROW] + t * npos,
-                             &sh.q_full);
+              for (int h = 0; h < C::NH; ++h)
+                ptx::tma_load_3d(sQ + t * C::Q_BYTES + h * C::BLK, &tm_q, h * 64, U[U_KVH] * G,
+                                 U[U_QROW] + t * npos, &sh.q_full);
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
         const int32_t npages = U[U_AN] + U[U_BN];
         const int32_t t0 = U[U_T0];
         const int32_t ntiles = U[U_NTILES];
         const int64_t toff = U[U_TOFF];
-        bool ok = true;
+        int32_t batch = -1, my_pid = -1;   // page id of list position 32 * batch + lane (-1: none)
+        int ok = 1;
         for (int32_t j = t0; j < t0 + ntiles && ok; ++j) {
+          const int32_t x0 = j * C::PPT;     // a tile's PPT positions never straddle a batch of 32
+          if ((x0 >> 5) != batch) {
+            batch = x0 >> 5;
+            const int32_t x = (batch << 5) + lane;
+            my_pid = -1;
+            if (x < npages) {
+              const int32_t idx = unit_table_index(U, x);
+              my_pid = 0;
+              if (idx < 0 || idx >= U[U_TOTAL] || toff + idx >= p.page_table_len) {
+                if (status) atomicOr(status, kStatusUnit);
+              } else {
+                my_pid = p.page_table[toff + idx];
+                if (my_pid < 0 || my_pid >= p.num_pages) {
+                  if (status) atomicOr(status, kStatusPageId);
+                  my_pid = 0;
+                }
+              }
+            }
+          }
           int32_t pages[C::PPT];
           int32_t n_ok = 0;
 #pragma unroll
           for (int c = 0; c < C::PPT; ++c) {
-            const int32_t x = j * C::PPT + c;
-            pages[c] = -1;
-            if (x < npages) {
-              const int32_t idx = unit_table_index(U, x);
-              int32_t pid = 0;
-              if (idx < 0 || idx >= U[U_TOTAL] || toff + idx >= p.page_table_len) {
-                if (status) atomicOr(status, kStatusUnit);
-              } else {
-                pid = p.page_table[toff + idx];
-                if (pid < 0 || pid >= p.num_pages) {
-                  if (status) atomicOr(status, kStatusPageId);
-                  pid = 0;
-                }
+            pages[c] = __shfl_sync(0xffffffffu, my_pid, (x0 + c) & 31);
+            n_ok += pages[c] >= 0 ? 1 : 0;
+          }
+          if (lane == 0) {
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {  // K then V
+              const uint32_t item = kv_item + which;
+              const int s = item % C::NSLOT;
+              if (!ptx::mbar_wait(&sh.kv_empty[s], ((item / C::NSLOT) & 1) ^ 1, abort, status, kStatusTimeout)) {
+                ok = 0;
+                break;
               }
-              pages[c] = pid;
-              ++n_ok;
+              ptx::mbar_arrive_expect_tx(&sh.kv_full[s], (uint32_t)(n_ok * P * D * 2));
+              uint8_t* dst = sKV + s * C::TILE_BYTES;
+#pragma unroll
+              for (int c = 0; c < C::PPT; ++c) {
+                if (pages[c] < 0) continue;
+#pragma unroll
+                for (int h = 0; h < C::NH; ++h)
+                  ptx::tma_load_3d(dst + h * C::BLK + c * P * 128, which ? &tm_v : &tm_k, h * 64, 0, pages[c],
+                                   &sh.kv_full[s]);
+              }
             }
           }
-#pragma unroll
-          for (int which = 0; which < 2; ++which) {  // K then V
-            const int s = kv_item % C::NSLOT;
-            if (!ptx::mbar_wait(&sh.kv_empty[s], ((kv_item / C::NSLOT) & 1) ^ 1, abort, status, kStatusTimeout)) {
-              ok = false;
-              break;
-            }
-            ptx::mbar_arrive_expect_tx(&sh.kv_full[s], (uint32_t)(n_ok * P * D * 2));
-            uint8_t* dst = sKV + s * C::TILE_BYTES;
-#pragma unroll
-            for (int c = 0; c < C::PPT; ++c) {
-              if (pages[c] < 0) continue;
-#pragma unroll
-              for (int h = 0; h < C::NH; ++h)
-                ptx::tma_load_3d(dst + h * C::BLK + c * P * 128, which ? &tm_v : &tm_k, h * 64, 0, pages[c],
-                                 &sh.kv_full[s]);
-            }
-            ++kv_item;
-          }
+          kv_item += 2;
+          ok = __shfl_sync(0xffffffffu, ok, 0);
         }
         if (!ok) break;
       }
