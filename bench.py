@@ -43,7 +43,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference", "dense"],
+                    help="ours: the SegPaged library; reference: the fp64 oracle on the host cores; dense: "
+                         "the dense-layout baseline (PyTorch SDPA, all heads at full context, explicit mask)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle sample")
@@ -292,6 +294,76 @@ def run_reference(args, rank, world):
     return 0
 
 
+def run_dense(args, rank, world, local):
+    """Dense-layout baseline on the same GPU: every head keeps its full context as a dense [Hq, L, D] K/V and
+    the sink-plus-window visibility is an explicit boolean mask given to PyTorch's scaled_dot_product_attention
+    (the masked slow path SegPagedAttention avoids). One layer of each kind is timed with CUDA events: query
+    rows are chunked so each mask stays near 2 GB, each chunk's mask is built before its call, and only the
+    attention calls are timed, each between its own events. Per-layer times are weighted by how many layers
+    of that kind the workload has."""
+    if rank != 0:
+        return 0
+    import torch
+    import torch.nn.functional as F
+    from head_sparse_paged_b200 import synth
+    from head_sparse_paged_b200.runner import visible_flops
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = rank_workload(args.workload, 0)
+    kinds = {}
+    for li in range(w.layers):
+        kinds.setdefault(int(w.classes[li][..., 0].sum()), []).append(li)
+    G, D = w.group, w.head_dim
+    scale = 1.0 / math.sqrt(D)
+    per_layer_ms, ms_step = {}, 0.0
+    _, k_all, v_all = synth.layer_inputs(w, 0, device=device)
+    cq, ck = w.cu_q(), w.cu_k()
+    for key, lis in kinds.items():
+        li = lis[0]
+        q = synth.layer_inputs(w, li, device=device, parts="q")[0]
+        if w.layers == 1:
+            _, k_all, v_all = synth.layer_inputs(w, li, device=device)
+        ms_layer = 0.0
+        for b in range(w.num_seqs):
+            L, Lq = w.ctx_lens[b], w.q_lens[b]
+            if Lq == 0:
+                continue
+            kk = k_all[ck[b]:ck[b + 1]].transpose(0, 1).repeat_interleave(G, dim=0)[None]   # [1, Hq, L, D]
+            vv = v_all[ck[b]:ck[b + 1]].transpose(0, 1).repeat_interleave(G, dim=0)[None]
+            qq = q[cq[b]:cq[b + 1]].transpose(0, 1)[None]                                      # [1, Hq, Lq, D]
+            cls = torch.from_numpy(w.classes[li, b]).to(device).repeat_interleave(G, dim=0)  # [Hq, 3]
+            glob, S, W = cls[:, 0, None, None] != 0, cls[:, 1, None, None], cls[:, 2, None, None]
+            j = torch.arange(L, device=device)[None, None, :]
+            chunk = max(1, int(2e9 // (w.num_q_heads * L)))
+            pairs = []
+            for rep in range(2):          # the first pass warms up; only the second is timed
+                for r0 in range(0, Lq, chunk):
+                    i = (L - Lq + torch.arange(r0, min(r0 + chunk, Lq), device=device))[None, :, None]
+                    m = ((j <= i) & (glob | (j < S) | (j > i - W)))[None]
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    F.scaled_dot_product_attention(qq[:, :, r0:r0 + m.shape[2]], kk, vv, attn_mask=m, scale=scale)
+                    e1.record()
+                    if rep == 1:
+                        pairs.append((e0, e1))
+                    del m
+            torch.cuda.synchronize()
+            ms_layer += sum(a.elapsed_time(b_) for a, b_ in pairs)
+            del kk, vv
+        per_layer_ms[f"{len(lis)} layers with {key} global heads"] = ms_layer
+        ms_step += ms_layer * len(lis)
+    flops = visible_flops(w)
+    line = {
+        "impl": "dense", "metric": METRIC, "value": flops / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": 1, "ms_per_step": ms_step, "ms_per_layer": ms_step / w.layers, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic", "config": workload_config(w), "dense_ms_by_layer_kind": per_layer_ms,
+        "note": "PyTorch SDPA with an explicit boolean mask over dense K/V of every head at full context; "
+                "value = visible FLOPs / time, so it is directly comparable with the SegPaged line",
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def workload_config(w):
     return {"workload": w.name, "description": w.description, "layers": w.layers, "seq_lens": list(w.ctx_lens),
             "q_lens": list(w.q_lens), "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
@@ -453,6 +525,8 @@ def main(argv=None):
     rank, world, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.impl == "dense":
+        return run_dense(args, rank, world, local)
     if world > 1:
         import datetime
         import torch
