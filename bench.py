@@ -419,7 +419,12 @@ def run_ours(args, rank, world, local):
     value = world * flops_step * args.steps / (ms_total * 1e-3) / 1e12
     achieved = sum(flops_layer[li] * len(prefill_ms[li]) for li in prefill_ms) / (prefill_total_ms * 1e-3) / 1e12
     peaks, src = load_peaks()
-    peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    # A kernel timed inside a long run (or one that hit the power cap) is held to the sustained GEMM peak,
+    # a short burst at full clocks to the burst peak.
+    clocks = clk.summary()
+    sustained = ms_total >= 1000.0 or "sw_power_cap" in (clocks.get("reasons") or [])
+    tf_name = "bf16_tflops_sustained" if sustained and "bf16_tflops_sustained" in peaks else "bf16_tflops"
+    peak_tf = float(peaks[tf_name])
     peak_bw = float(peaks.get("hbm_gbs"))
     traffic = traffic_per_launch(w.name)
     # algorithmic bytes of each prefill launch: stored K/V pages read once, Q read, O and LSE written
@@ -433,7 +438,7 @@ def run_ours(args, rank, world, local):
         peak_name = "hbm_gbs"
     else:
         bound, unit, peak = "tensor", "TFLOP/s", peak_tf
-        peak_name = "bf16_tflops_sustained"
+        peak_name = tf_name
     kinds = {}
     for li in runner.layers:
         kinds.setdefault("all-global" if runner.state[li].cls[..., 0].all() else "mixed", []).append(li)
@@ -477,7 +482,7 @@ def run_ours(args, rank, world, local):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps * n_layers * 2,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
     print(json.dumps(line))
     return 0

@@ -12,20 +12,21 @@
 // Per CTA, 12 warps (3 warpgroups):
 //   warps 0-3   softmax for query tile 0, warps 4-7 softmax for query tile 1: one tile row per thread.
 //               tcgen05.ld of the S row, per-row bounds only on edge tiles, row max (3-input max),
-//               lazy O rescale (only when the running max grows by more than 2^8), exp2 -- three of
-//               every four element pairs on the MUFU unit, the fourth on the FMA pipe by a cubic --,
-//               row sum and scaling in packed f32x2 arithmetic, P written back to TMEM as bf16 over S,
-//               and the epilogue (O / l -> bf16, LSE = ln 2 * (m + log2 l)).
-//   warp 8      producer: claims units, TMA-loads both Q tiles (3-D map over [rows, Hq, D], box
+//               lazy O rescale (only when the running max grows by more than 2^8), exp2 on the MUFU
+//               unit, row sum and scaling in packed f32x2 arithmetic, P written back to TMEM as bf16 over
+//               S and published in two halves of 64 keys, and the epilogue (O / l -> bf16,
+//               LSE = ln 2 * (m + log2 l)).
+//   warp 8      producer (whole warp: page-table lookups; lane 0: barriers and TMA): claims units, TMA-loads both Q tiles (3-D map over [rows, Hq, D], box
 //               64 x G x 128/G) and, for every 128-key tile, the K and V pages (3-D map over
 //               [pages, P, D], coordinate = physical page id) into 128B-swizzled shared-memory slots.
-//   warp 9      MMA issuer, in the order PV0(j-1), S0(j), PV1(j-1), S1(j): S_t = Q_t K^T
+//   warp 9      MMA issuer (whole warp, one elected lane issues), in the order PV0(j-1), S0(j), PV1(j-1), S1(j): S_t = Q_t K^T
 //               (tcgen05.mma, both operands in shared memory, f32 in TMEM) and O_t += P_t V (P from
-//               TMEM, V MN-major from shared memory). The commit that publishes S_t(j) also covers
-//               PV_t(j-1), so when a softmax warp sees S_t(j) its O_t is stable and can be rescaled.
+//               TMEM, V MN-major from shared memory; keys 0-63 as soon as that half of P is written).
+//               The commit that publishes S_t(j) also covers PV_t(j-1), so when a softmax warp sees
+//               S_t(j) its O_t is stable and can be rescaled.
 //   warps 10-11 idle.
-// Every wait is bounded: on a timeout the CTA raises its abort flag, reports
-// SEGPAGED_STATUS_TIMEOUT, drains the MMA pipe and frees its tensor memory before returning.
+// Every wait is bounded: on a timeout the CTA raises its abort flag, reports SEGPAGED_STATUS_TIMEOUT,
+// waits (bounded) for its TMA copies and MMAs in flight, and frees its tensor memory before returning.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -80,7 +81,7 @@ struct PrefillParams {
 struct PrefillShared {
   uint64_t unit_full[2], unit_empty[2];
   uint64_t q_full, q_empty;
-  uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+  uint64_t s_full[2], p_half[2], p_full[2], o_full[2], o_free[2];
   uint64_t mma_drain;
   uint64_t kv_full[10], kv_empty[10];
   __align__(16) int32_t unit[2][U_NFIELDS];
@@ -127,33 +128,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair, on the FMA and integer pipes: n = round(x) through the 1.5 * 2^23 rounding trick,
-// f = x - n in [-1/2, 1/2], 2^f by a cubic minimising relative error (coefficients from
-// csrc/fit_exp2_poly.py, max relative error 7.5e-5), then n is added to the exponent bits. x is
-// clamped to >= -126 so the exponent never wraps; masked logits (-inf) then give ~1e-38 instead of 0.
-__device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t x2) {
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  x0 = fmaxf(x0, -126.0f);
-  x1 = fmaxf(x1, -126.0f);
-  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t nmagic = f2_pack(-12582912.0f, -12582912.0f);
-  const uint64_t xc = f2_pack(x0, x1);
-  const uint64_t t = f2_add(xc, magic);                  // low mantissa bits hold round(x)
-  const uint64_t n = f2_add(t, nmagic);                  // round(x) as a float
-  const uint64_t neg1 = f2_pack(-1.0f, -1.0f);
-  const uint64_t f = f2_fma(n, neg1, xc);                // x - round(x)
-  uint64_t p = f2_fma(f2_pack(0x1.c3f76p-5f, 0x1.c3f76p-5f), f, f2_pack(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
-  p = f2_fma(p, f, f2_pack(0x1.62f31ap-1f, 0x1.62f31ap-1f));
-  p = f2_fma(p, f, f2_pack(0x1.fff692p-1f, 0x1.fff692p-1f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
-  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
-  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
-}
-
 template <int D, int P>
 __global__ void __launch_bounds__(384, 1)
     segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -174,6 +148,7 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_init(&sh.unit_full[i], 1);
       ptx::mbar_init(&sh.unit_empty[i], 9);   // MMA lane 0 + 8 softmax warps
       ptx::mbar_init(&sh.s_full[i], 1);
+      ptx::mbar_init(&sh.p_half[i], 4);
       ptx::mbar_init(&sh.p_full[i], 4);
       ptx::mbar_init(&sh.o_full[i], 1);
       ptx::mbar_init(&sh.o_free[i], 4);
@@ -216,6 +191,8 @@ __global__ void __launch_bounds__(384, 1)
       // The whole warp walks the schedule; lane 0 does the barrier and TMA work, and the 32 lanes fetch
       // the page-table entries of 32 list positions at once, so a tile's loads never wait on a lookup.
       uint32_t kv_item = 0;
+      uint32_t kv_issued = 0;        // lane 0: KV items whose loads were issued
+      int32_t q_ring = -1;           // lane 0: ring index of the last query-tile load issued
       for (uint32_t ring = 0;; ++ring) {
         const int slot = ring & 1;
         int go = 1;
@@ -241,6 +218,7 @@ __global__ void __launch_bounds__(384, 1)
           if (go) {
             const int nq = U[U_HALF] ? 1 : 2;   // a half unit has no rows in its second query tile
             ptx::mbar_arrive_expect_tx(&sh.q_full, nq * C::Q_BYTES);
+            q_ring = (int32_t)ring;
             for (int t = 0; t < nq; ++t)
 #pragma unroll
               for (int h = 0; h < C::NH; ++h)
@@ -301,6 +279,7 @@ __global__ void __launch_bounds__(384, 1)
                   ptx::tma_load_3d(dst + h * C::BLK + c * P * 128, which ? &tm_v : &tm_k, h * 64, 0, pages[c],
                                    &sh.kv_full[s]);
               }
+              kv_issued = item + 1;
             }
           }
           kv_item += 2;
@@ -308,83 +287,106 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
       }
-    } else if (warp == 9 && lane == 0) {
+      // After giving up, wait (bounded, ignoring the abort flag) for the copies this warp issued, so
+      // none lands in shared memory after the CTA has exited.
+      if (lane == 0 && *abort) {
+        const uint32_t first = kv_issued > (uint32_t)C::NSLOT ? kv_issued - C::NSLOT : 0u;
+        for (uint32_t it = first; it < kv_issued; ++it)
+          ptx::mbar_wait(&sh.kv_full[it % C::NSLOT], (it / C::NSLOT) & 1, nullptr, status, kStatusTimeout);
+        if (q_ring >= 0) ptx::mbar_wait(&sh.q_full, (uint32_t)q_ring & 1, nullptr, status, kStatusTimeout);
+      }
+      __syncwarp();
+    } else if (warp == 9) {
       // -------------------------------------------------------------------------- MMA issuer
+      // The whole warp walks the schedule, so barrier parities, slots and descriptors are warp-uniform
+      // values; one elected lane issues each tcgen05.mma and tcgen05.commit.
+      const uint32_t leader = ptx::elect_one();
       const uint32_t q_base = ptx::smem_addr(sQ), kv_base = ptx::smem_addr(sKV);
       uint32_t kv_item = 0, act[2] = {0, 0}, pcount[2] = {0, 0};
       bool ok = true;
-      // O_t (+)= P_t V for the V tile in KV item vi; `first` starts the unit's accumulation.
+      auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kStatusTimeout));
+      };
+      // O_t (+)= P_t V for the V tile in KV item vi; `first` starts the unit's accumulation. The softmax
+      // warps publish P_t in two halves of 64 keys: the first half's MMAs run while they finish the second.
       auto issue_pv = [&](int t, uint32_t vi, bool first) -> bool {
-        if (!ptx::mbar_wait(&sh.p_full[t], pcount[t] & 1, abort, status, kStatusTimeout)) return false;
-        ++pcount[t];
-        if (first && act[t] > 0 && !ptx::mbar_wait(&sh.o_free[t], (act[t] - 1) & 1, abort, status, kStatusTimeout))
-          return false;
+        if (!wait(&sh.p_half[t], pcount[t] & 1)) return false;
+        if (first && act[t] > 0 && !wait(&sh.o_free[t], (act[t] - 1) & 1)) return false;
         const int s = vi % C::NSLOT;
-        if (t == 0 && !ptx::mbar_wait(&sh.kv_full[s], (vi / C::NSLOT) & 1, abort, status, kStatusTimeout))
-          return false;
+        if (t == 0 && !wait(&sh.kv_full[s], (vi / C::NSLOT) & 1)) return false;
         ptx::tc_fence_after();
         const uint32_t pa = tmem + t * 128;                 // P_t: bf16 pairs over the first 64 columns of S_t
         const uint32_t od = tmem + 256 + t * D;
-        const uint32_t vb = kv_base + s * C::TILE_BYTES;
+        const uint64_t vdesc = ptx::sw128_desc(kv_base + s * C::TILE_BYTES, C::BLK, 1024);
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
-          ptx::umma_ts(od, pa + kk * 8, ptx::sw128_desc(vb + kk * 16 * 128, C::BLK, 1024), C::IDESC_O,
+        for (int kk = 0; kk < C::BN / 32; ++kk)             // 16 keys = 2048 B of V = 128 in the address field
+          ptx::umma_ts(leader, od, pa + kk * 8, vdesc + (uint64_t)(kk * 128), C::IDESC_O,
                        (kk > 0 || !first) ? 1u : 0u);
+        if (!wait(&sh.p_full[t], pcount[t] & 1)) return false;
+        ++pcount[t];
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = C::BN / 32; kk < C::BN / 16; ++kk)
+          ptx::umma_ts(leader, od, pa + kk * 8, vdesc + (uint64_t)(kk * 128), C::IDESC_O, 1u);
         return true;
       };
       auto issue_s = [&](int t, uint32_t kb) {
-        const uint32_t qa = q_base + t * C::Q_BYTES;
         const uint32_t sd = tmem + t * 128;
+        const uint64_t qdesc = ptx::sw128_desc(q_base + t * C::Q_BYTES, 16, 1024);
+        const uint64_t kdesc = ptx::sw128_desc(kb, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-          ptx::umma_ss(sd, ptx::sw128_desc(qa + off, 16, 1024), ptx::sw128_desc(kb + off, 16, 1024), C::IDESC_S,
-                       kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * C::BLK + (kk & 3) * 32) >> 4);
+          ptx::umma_ss(leader, sd, qdesc + off, kdesc + off, C::IDESC_S, kk > 0 ? 1u : 0u);
         }
-        ptx::umma_commit(&sh.s_full[t]);
+        ptx::umma_commit(leader, &sh.s_full[t]);
       };
       for (uint32_t ring = 0; ok; ++ring) {
         const int slot = ring & 1;
-        if (!ptx::mbar_wait(&sh.unit_full[slot], (ring >> 1) & 1, abort, status, kStatusTimeout)) { ok = false; break; }
+        if (!wait(&sh.unit_full[slot], (ring >> 1) & 1)) { ok = false; break; }
         const int32_t ntiles = sh.unit[slot][U_NTILES];
         const bool two = sh.unit[slot][U_HALF] == 0;   // second query tile active
-        ptx::mbar_arrive(&sh.unit_empty[slot]);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
         if (ntiles < 0) break;
-        if (!ptx::mbar_wait(&sh.q_full, (ring & 1), abort, status, kStatusTimeout)) { ok = false; break; }
+        if (!wait(&sh.q_full, (ring & 1))) { ok = false; break; }
         uint32_t prev_vi = 0;
         for (int32_t j = 0; j < ntiles && ok; ++j) {
           const uint32_t ki = kv_item, vi = kv_item + 1;
           kv_item += 2;
           if (j > 0 && !issue_pv(0, prev_vi, j == 1)) { ok = false; break; }
           const int s = ki % C::NSLOT;
-          if (!ptx::mbar_wait(&sh.kv_full[s], (ki / C::NSLOT) & 1, abort, status, kStatusTimeout)) { ok = false; break; }
+          if (!wait(&sh.kv_full[s], (ki / C::NSLOT) & 1)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t kb = kv_base + s * C::TILE_BYTES;
           issue_s(0, kb);
           if (j > 0) {
             if (two && !issue_pv(1, prev_vi, j == 1)) { ok = false; break; }
-            ptx::umma_commit(&sh.kv_empty[prev_vi % C::NSLOT]);
+            ptx::umma_commit(leader, &sh.kv_empty[prev_vi % C::NSLOT]);
           }
           if (two) issue_s(1, kb);
-          ptx::umma_commit(&sh.kv_empty[s]);
-          if (j == ntiles - 1) ptx::umma_commit(&sh.q_empty);
+          ptx::umma_commit(leader, &sh.kv_empty[s]);
+          if (j == ntiles - 1) ptx::umma_commit(leader, &sh.q_empty);
           prev_vi = vi;
         }
         if (!ok) break;
         // the unit's last PV of each tile publishes its O
         if (!issue_pv(0, prev_vi, ntiles == 1)) break;
-        ptx::umma_commit(&sh.o_full[0]);
+        ptx::umma_commit(leader, &sh.o_full[0]);
         if (two) {
           if (!issue_pv(1, prev_vi, ntiles == 1)) break;
-          ptx::umma_commit(&sh.o_full[1]);
+          ptx::umma_commit(leader, &sh.o_full[1]);
         }
-        ptx::umma_commit(&sh.kv_empty[prev_vi % C::NSLOT]);
+        ptx::umma_commit(leader, &sh.kv_empty[prev_vi % C::NSLOT]);
         ++act[0];
         if (two) ++act[1];
       }
-      // Drain: every MMA this CTA issued has completed before tensor memory is released.
-      ptx::umma_commit(&sh.mma_drain);
-      ptx::mbar_wait(&sh.mma_drain, 0, abort, status, kStatusTimeout);
+      // Drain: every MMA this CTA issued has completed before tensor memory is released (a bounded wait
+      // that ignores the abort flag).
+      __syncwarp();
+      ptx::umma_commit(leader, &sh.mma_drain);
+      ptx::mbar_wait(&sh.mma_drain, 0, nullptr, status, kStatusTimeout);
+      __syncwarp();
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
@@ -423,10 +425,30 @@ __global__ void __launch_bounds__(384, 1)
       const bool is_global = u[U_GLOBAL] != 0;
       const int32_t S = u[U_SINK], W = u[U_WIN];
       const int32_t npages = u[U_AN] + u[U_BN];
+      const int32_t an = u[U_AN], b0 = u[U_B0], nsink = u[U_NSINK], w0 = u[U_W0];
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
 
       for (int32_t j = 0; j < ntiles; ++j) {
+        // Logical page of every slot of this KV tile, worked out before S is ready; a row needs per-column
+        // bounds only if some key of the tile is invisible to it (causal edge, window edge, sink tail, or
+        // a short last tile).
+        int32_t lp[C::PPT];
+        bool need_mask = false;
+#pragma unroll
+        for (int c = 0; c < C::PPT; ++c) {
+          const int32_t x = (t0 + j) * C::PPT + c;
+          if (x < npages) {
+            const int32_t idx = x < an ? x : b0 + (x - an);
+            lp[c] = idx < nsink ? idx : w0 + (idx - nsink);
+            const int32_t j0 = lp[c] * P, j1 = j0 + P - 1;
+            const bool all_vis = (j1 <= i_pos) && (is_global || j1 < S || j0 > i_pos - W);
+            need_mask |= !all_vis;
+          } else {
+            lp[c] = -1;
+            need_mask = true;
+          }
+        }
         if (!wwait(&sh.s_full[tile], scount & 1)) { ok = false; break; }
         ++scount;
         ptx::tc_fence_after();
@@ -438,23 +460,6 @@ __global__ void __launch_bounds__(384, 1)
         ptx::tmem_ld32(sbuf + 64, reinterpret_cast<uint32_t*>(s) + 64);
         ptx::tmem_ld32(sbuf + 96, reinterpret_cast<uint32_t*>(s) + 96);
 
-        // Logical page of every slot of this KV tile; a row needs per-column bounds only if some key
-        // of the tile is invisible to it (causal edge, window edge, sink tail, or a short last tile).
-        int32_t lp[C::PPT];
-        bool need_mask = false;
-#pragma unroll
-        for (int c = 0; c < C::PPT; ++c) {
-          const int32_t x = (t0 + j) * C::PPT + c;
-          if (x < npages) {
-            lp[c] = unit_logical_page(u, unit_table_index(u, x));
-            const int32_t j0 = lp[c] * P, j1 = j0 + P - 1;
-            const bool all_vis = (j1 <= i_pos) && (is_global || j1 < S || j0 > i_pos - W);
-            need_mask |= !all_vis;
-          } else {
-            lp[c] = -1;
-            need_mask = true;
-          }
-        }
         // Row max as eight independent 3-input max chains per half, so no long dependency chain.
         float mh[8];
 #pragma unroll
@@ -505,53 +510,50 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t nmu2 = f2_pack(-mu, -mu);
         uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {          // two halves of 64 columns -> 32 packed P columns each
+        for (int h = 0; h < 2; ++h) {          // two halves of 64 keys -> 32 packed P columns each
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int e = h * 64 + 2 * c;
             const uint64_t x2 = f2_fma(f2_pack(s[e], s[e + 1]), sl2_2, nmu2);
-            uint64_t p2;
-            if ((c & 3) == 3) {
-              p2 = exp2_poly_pair(x2);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              p2 = f2_pack(ptx::ex2(x0), ptx::ex2(x1));
-            }
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const uint64_t p2 = f2_pack(ptx::ex2(x0), ptx::ex2(x1));
             sum2[c & 3] = f2_add(sum2[c & 3], p2);
             float p0, p1;
             f2_unpack(p2, p0, p1);
             pk[c] = ptx::pack_bf16x2(p0, p1);
           }
           ptx::tmem_st32(sbuf + h * 32, pk);
-        }
-        if (__any_sync(0xffffffffu, resc)) {
-          // Rescale O_t in place now that S is dead. O_t holds every PV issued so far (the commit that
-          // published S_t(j) covered PV_t(j-1)), and PV_t(j) waits for this warp's p_full arrival.
-          const uint64_t a2 = f2_pack(alpha, alpha);
+          if (h == 0 && __any_sync(0xffffffffu, resc)) {
+            // Rescale O_t in place before any of P_t(j) is published (the first half of S is dead by now,
+            // which leaves registers for it). O_t holds every PV issued so far -- the commit that published
+            // S_t(j) covered PV_t(j-1) -- and PV_t(j) waits for this warp's arrivals.
+            const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(obuf + c * 32, r);
-            ptx::tmem_ld_wait();
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              ptx::tmem_ld32(obuf + c * 32, r);
+              ptx::tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              float lo, hi;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), a2), lo, hi);
-              r[2 * k] = __float_as_uint(lo);
-              r[2 * k + 1] = __float_as_uint(hi);
+              for (int k = 0; k < 16; ++k) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), a2), lo, hi);
+                r[2 * k] = __float_as_uint(lo);
+                r[2 * k + 1] = __float_as_uint(hi);
+              }
+              ptx::tmem_st32(obuf + c * 32, r);
             }
-            ptx::tmem_st32(obuf + c * 32, r);
           }
+          // publish this half of P_t(j): the first lets the MMA warp start on keys 0-63
+          ptx::tmem_st_wait();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(h == 0 ? &sh.p_half[tile] : &sh.p_full[tile]);
         }
         float sa, sb;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
         l_run += sa + sb;
-        ptx::tmem_st_wait();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.p_full[tile]);
       }
       if (!ok) break;
 
