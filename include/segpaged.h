@@ -214,6 +214,61 @@ int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const void* q, int3
                                   const segpaged_unit* units_host, int64_t num_units, float softmax_scale, void* o,
                                   float* lse, int32_t* status, void* stream);
 
+/* ------------------------------------------------------------------------------------------------
+ * Token importance for sparse FFN.
+ *
+ * The pages run the dense FFN only on the top-k tokens by attention score and send the other tokens
+ * down the residual identity path, choosing them from the attention signal of the prefill
+ * ("RedKnot – 小红书研发并开源的长上下文大模型推理引擎" (shshi.cn), 技术原理 3 "稀疏FFN动态调度";
+ * "为什么长上下文推理这么慢？RedKnot…" (bjdmk.com.cn), 二 "三大核心机制" item 2 "稀疏 FFN 与自适应专家
+ * Top-K"; zhichai.net, 事件内容 item 2 "稀疏 FFN"). They define neither the score nor the tie rule. The
+ * reading taken here: the score of a token of the query range is the attention mass it receives in
+ * this prefill,
+ *   mass[r] = sum over query heads h and query positions i of exp(s_hij - LSE_hi) for j in V_h(i),
+ * where j is the position of query row r (its own key), s the scaled logits of the prefill and LSE
+ * its row log-sum-exp. The FFN itself (model weights) is not part of this library.
+ * ------------------------------------------------------------------------------------------------ */
+
+/* One work item of a mass plan: a (sequence, KV head, 128-key tile of the query range) and the query
+ * tiles that can see it. Produced by segpaged_mass_plan; the fields are private. 64 bytes. */
+typedef struct {
+  int32_t v[16];
+} segpaged_mass_item;
+
+/* Plans segpaged_token_mass (host only). Inputs as for segpaged_prefill_plan. Writes the items to
+ * `items` (host, capacity entries; NULL to only count) and returns their number, or an error
+ * (SEGPAGED_ERR_CAPACITY if capacity is too small). */
+int64_t segpaged_mass_plan(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                           const segpaged_head_class* cls, const int32_t* page_table_offs,
+                           segpaged_mass_item* items, int64_t capacity);
+
+/* Device workspace segpaged_token_mass needs: one partial sum per (KV head, query row) and a counter. */
+size_t segpaged_mass_workspace_bytes(const segpaged_dims* dims, int32_t total_q);
+
+/*
+ * mass[r] for every query row r (dev, float32 [total_q]), as defined above. Recomputes the logits of
+ * every (query tile, key tile) pair whose keys lie in the query range on the tensor cores and
+ * normalises them with `lse`, the natural-log LSE [Hq, total_q] (dev, float32) that
+ * segpaged_attn_prefill wrote for the same q, pools and scale. Same q, pools, page table and scale
+ * as that prefill. items (dev) [num_items] from segpaged_mass_plan; workspace (dev, 256-byte
+ * aligned) of segpaged_mass_workspace_bytes. The sum over KV heads is taken in a fixed order, so
+ * the result does not depend on scheduling or on the physical page ids. Asynchronous on `stream`.
+ */
+int segpaged_token_mass(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
+                        const int32_t* page_table, int64_t page_table_len, const segpaged_mass_item* items,
+                        int64_t num_items, const float* lse, float softmax_scale, float* mass, void* workspace,
+                        size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * Top-k tokens of each sequence by mass (all device memory): for sequence b, the k_b = min(max(
+ * k_per_seq[b], 0), Lq_b) rows of [cu_seqlens_q[b], cu_seqlens_q[b+1]) with the largest mass; among
+ * equal values the lower row wins. The chosen global row indices are written in ascending order to
+ * selected[off_b .. off_b + k_b), off_b = sum of k_c over c < b (size `selected` for the sum of all
+ * k_b). mass must be finite and >= 0 (as segpaged_token_mass writes it). One block per sequence.
+ */
+int segpaged_select_topk(int32_t num_seqs, const float* mass, const int32_t* cu_seqlens_q, const int32_t* k_per_seq,
+                         int32_t* selected, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

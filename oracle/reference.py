@@ -21,6 +21,11 @@ Everything here is written from the method's definition, in fp64 where it is flo
   ("RoPE位置对齐", shshi.cn, "RedKnot技术原理" 2 "位置无关缓存复用").
 * ``rope_cos_sin`` / ``rope_rotate_bf16`` -- the RoPE delta rotation, rotate-half pairing
   (d, d + D/2), with the bit-exact fp32 rule stated in their docstrings.
+* ``token_mass`` / ``select_topk`` -- the token score of the sparse-FFN selection (top-k tokens by
+  attention score run the dense FFN, the rest take the residual path: shshi.cn, "RedKnot技术原理" 3
+  "稀疏FFN动态调度"). The pages define neither the score nor ties; the reading used here: a token's
+  score is the attention mass it receives from every query row and head of the prefill, and among
+  equal scores the lower row is chosen.
 
 ``OracleLib`` wraps the C oracle (segpaged_oracle.c), which forms the visible set by brute-force
 predicate scan instead of ranges; the tests require both to agree.
@@ -123,6 +128,38 @@ def attention(pb: Problem, scale: float, rows=None):
     for t, (r, h) in enumerate(rows):
         o[t], lse[t], _, _ = attention_row(pb, r, h, scale)
     return o, lse
+
+
+def token_mass(pb: Problem, scale: float) -> np.ndarray:
+    """Attention mass received by each query row's own token, fp64 [total_q].
+
+    mass[r] = sum over query heads h and query rows r' (position i) of p_h(i, j) for j in V_h(i),
+    j the position of row r, p the softmax probabilities of ``attention_row``.
+    """
+    mass = np.zeros(pb.q.shape[0])
+    for rr in range(pb.q.shape[0]):
+        b, _ = pb.row_seq_pos(rr)
+        L = int(pb.cu_k[b + 1] - pb.cu_k[b])
+        q0 = L - int(pb.cu_q[b + 1] - pb.cu_q[b])
+        for h in range(pb.Hq):
+            _, _, p, vis = attention_row(pb, rr, h, scale)
+            keep = vis >= q0
+            np.add.at(mass, int(pb.cu_q[b]) + (vis[keep] - q0), p[keep])
+    return mass
+
+
+def select_topk(mass: np.ndarray, cu_q, k_per_seq) -> np.ndarray:
+    """Global rows chosen per sequence, concatenated in sequence order, each list ascending.
+
+    Sequence b keeps min(max(k_b, 0), Lq_b) rows of largest mass; equal masses prefer the lower row.
+    """
+    out = []
+    for b in range(len(cu_q) - 1):
+        lo, hi = int(cu_q[b]), int(cu_q[b + 1])
+        kb = min(max(int(k_per_seq[b]), 0), hi - lo)
+        rows = sorted(range(lo, hi), key=lambda r: (-mass[r], r))[:kb]
+        out.extend(sorted(rows))
+    return np.asarray(out, dtype=np.int64)
 
 
 # ----------------------------------------------------------------------------------------------
@@ -250,6 +287,8 @@ class OracleLib:
         self.lib.oracle_attention.argtypes = [ctypes.c_int] * 4 + [p] * 8 + [p, ctypes.c_int64, ctypes.c_double, p, p, p]
         self.lib.oracle_probs.restype = ctypes.c_int64
         self.lib.oracle_probs.argtypes = [ctypes.c_int] * 4 + [p] * 7 + [ctypes.c_int64, ctypes.c_int64, ctypes.c_double, p]
+        self.lib.oracle_token_mass.restype = ctypes.c_int
+        self.lib.oracle_token_mass.argtypes = [ctypes.c_int] * 4 + [p] * 7 + [ctypes.c_double, p]
 
     @staticmethod
     def _ptr(a):
@@ -299,3 +338,14 @@ class OracleLib:
         if n < 0:
             raise ValueError("oracle_probs: malformed item")
         return p[:L], int(n)
+
+    def token_mass(self, pb: Problem, scale: float) -> np.ndarray:
+        """Attention mass received by each query row's token, fp64 [total_q] (brute-force visible set)."""
+        a = self._common(pb)
+        m = np.zeros(max(pb.q.shape[0], 1), dtype=np.float64)
+        rc = self.lib.oracle_token_mass(pb.B, pb.Hq, pb.Hkv, pb.D, self._ptr(a["cu_q"]), self._ptr(a["cu_k"]),
+                                        self._ptr(a["g"]), self._ptr(a["s"]), self._ptr(a["w"]),
+                                        self._ptr(a["q"]), self._ptr(a["k"]), float(scale), self._ptr(m))
+        if rc != 0:
+            raise ValueError("oracle_token_mass failed")
+        return m[: pb.q.shape[0]]

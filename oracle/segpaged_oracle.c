@@ -131,3 +131,68 @@ int64_t oracle_probs(int B, int Hq, int Hkv, int D, const int32_t* cu_q, const i
   for (int64_t j = 0; j < L; ++j) p_out[j] = (p_out[j] == -INFINITY) ? 0.0 : exp(p_out[j] - mx) / sum;
   return n;
 }
+
+/*
+ * Attention mass each token of the query range receives in the prefill (the token score of the
+ * sparse-FFN selection: "RedKnot技术原理" 3 "稀疏FFN动态调度", shshi.cn; the reading of "attention
+ * score" as mass received is this project's, as the pages do not define it):
+ *
+ *   mass_out[r] = sum over query heads h and query rows r' of the same sequence, at position i,
+ *                 with j in V_h(i), of exp(s_hij - LSE_hi),
+ *
+ * where j is the position of query row r. Every LSE is formed first (two-pass, brute-force visible
+ * set), then every sum. Returns 0.
+ */
+int oracle_token_mass(int B, int Hq, int Hkv, int D, const int32_t* cu_q, const int32_t* cu_k,
+                      const int32_t* cls_global, const int32_t* cls_sink, const int32_t* cls_window,
+                      const float* q, const float* k, double scale, double* mass_out) {
+  const int G = Hq / Hkv;
+  for (int b = 0; b < B; ++b) {
+    const int64_t L = cu_k[b + 1] - cu_k[b], Lq = cu_q[b + 1] - cu_q[b], q0 = L - Lq;
+    if (Lq <= 0) continue;
+    double* lse = (double*)malloc(sizeof(double) * (size_t)(Lq * Hq));
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < Lq * Hq; ++t) {
+      const int64_t rr = t / Hq, h = t % Hq, i = q0 + rr;
+      const int kh = (int)(h / G);
+      const int cg = cls_global[b * Hkv + kh], cs = cls_sink[b * Hkv + kh], cw = cls_window[b * Hkv + kh];
+      const float* qrow = q + ((cu_q[b] + rr) * Hq + h) * (int64_t)D;
+      double mx = -INFINITY, sum = 0.0;
+      for (int pass = 0; pass < 2; ++pass)
+        for (int64_t j = 0; j < L; ++j) {
+          if (!oracle_visible(cg, cs, cw, i, j)) continue;
+          const float* krow = k + ((cu_k[b] + j) * Hkv + kh) * (int64_t)D;
+          double acc = 0.0;
+          for (int d = 0; d < D; ++d) acc += (double)qrow[d] * (double)krow[d];
+          const double s = scale * acc;
+          if (pass == 0) {
+            if (s > mx) mx = s;
+          } else {
+            sum += exp(s - mx);
+          }
+        }
+      lse[t] = mx + log(sum);
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < Lq; ++r) {
+      const int64_t j = q0 + r;
+      double m = 0.0;
+      for (int64_t rr = 0; rr < Lq; ++rr) {
+        const int64_t i = q0 + rr;
+        for (int h = 0; h < Hq; ++h) {
+          const int kh = h / G;
+          if (!oracle_visible(cls_global[b * Hkv + kh], cls_sink[b * Hkv + kh], cls_window[b * Hkv + kh], i, j))
+            continue;
+          const float* qrow = q + ((cu_q[b] + rr) * Hq + h) * (int64_t)D;
+          const float* krow = k + ((cu_k[b] + j) * Hkv + kh) * (int64_t)D;
+          double acc = 0.0;
+          for (int d = 0; d < D; ++d) acc += (double)qrow[d] * (double)krow[d];
+          m += exp(scale * acc - lse[rr * Hq + h]);
+        }
+      }
+      mass_out[cu_q[b] + r] = m;
+    }
+    free(lse);
+  }
+  return 0;
+}
