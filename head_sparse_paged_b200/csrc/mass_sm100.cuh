@@ -1,0 +1,390 @@
+// mass_sm100.cuh -- attention mass each query-range token receives in a prefill, on B200 (sm_100a).
+//
+// The sparse FFN keeps the dense FFN for the top-k tokens by attention score (shshi.cn, "RedKnot技术原理"
+// 3 "稀疏FFN动态调度"; bjdmk.com.cn, 二 item 2). The score read here is the mass a token receives:
+//   mass[r] = sum_h sum_i exp(s_hij - LSE_hi) over query rows i whose visible set V_h(i) holds j,
+// j the position of query row r. The row normalisers LSE come from the prefill, so this is a second
+// pass over the (query tile, key tile) pairs whose keys lie in the query range -- a small share of the
+// prefill's pairs when Lq << L.
+//
+// Work item: (sequence, KV head, 128-key tile x of the query range) and the query tiles that can see
+// it. Logits are computed transposed, S^T = K Q^T (tcgen05.mma, M = 128 keys, N = 128 query rows,
+// both operands K-major in 128B-swizzled shared memory, f32 in TMEM), so each thread of the mass
+// warpgroup owns one key's TMEM lane and sums its row: no cross-thread reduction. The sum of an item
+// goes to a per-(KV head, query row) partial; mass_reduce_kernel adds the KV heads in a fixed order.
+//
+// Per CTA, 6 warps:
+//   warps 0-3  mass: tcgen05.ld of the key's 128 logits, exp2(s * scale * log2 e - LSE_i * log2 e) with
+//              per-element bounds only on edge pairs, running sum in packed f32x2.
+//   warp 4     producer: claims items, TMA-loads the key tile's pages once and every query tile
+//              (same map as the prefill), and gathers the 128 rows' -LSE * log2 e into shared memory
+//              (+inf LSE for rows past the query range, so they contribute exp2(-inf) = 0).
+//   warp 5     MMA issuer (whole warp, one elected lane issues): S^T into one of two TMEM buffers.
+// Every wait is bounded, as in the prefill kernel.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "plan.h"
+#include "sm100_ptx.cuh"
+
+namespace segpaged {
+
+// Fields of a mass work item (segpaged_mass_item::v).
+enum MassField : int {
+  M_SEQ = 0,   // sequence b
+  M_KVH,       // KV head
+  M_TILE,      // logical key tile x: keys [128 x, 128 x + 128)
+  M_TOFF,      // offset of the (b, KV head) page-table entries
+  M_NSINK,     // stored sink pages (storage_split)
+  M_W0,        // first stored window page
+  M_GLOBAL,    // head class
+  M_SINK,
+  M_WIN,
+  M_Q0,        // first query position L - Lq
+  M_L,         // context length
+  M_QROW0,     // global row of the sequence's first query
+  M_T0,        // first query tile (of 128/G positions) that can see the key tile
+  M_NT,        // number of query tiles; -1 marks the end of the schedule
+  M_TOTAL,     // stored pages of the (b, KV head)
+  M_LQ,        // query positions of the sequence
+  M_NFIELDS
+};
+
+constexpr int32_t kMassStatusPageId = 1;
+constexpr int32_t kMassStatusTimeout = 4;
+constexpr int32_t kMassStatusUnit = 8;
+
+template <int D, int P>
+struct MassCfg {
+  static constexpr int NH = D / 64;                   // 128-byte swizzle column blocks across D
+  static constexpr int BLK = 128 * 128;               // bytes of one 64-column block of a 128-row tile
+  static constexpr int TILE_BYTES = 128 * D * 2;      // key tile or query tile
+  static constexpr int NQ = 3;                        // query-tile ring
+  static constexpr int PPT = 128 / P;                 // pages per key tile
+  static constexpr int SMEM_BYTES = TILE_BYTES * (1 + NQ) + NQ * 128 * 4 + 1024;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t TMEM_COLS = 256;          // two S^T buffers of 128 columns
+  static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, 128, 0, 0);
+};
+
+struct MassParams {
+  const int32_t* page_table;
+  int64_t page_table_len;
+  const int32_t* items;  // [num_items][M_NFIELDS]
+  int32_t num_items;
+  int32_t* counter;      // zeroed before the launch
+  int32_t* status;       // nullable
+  const float* lse;      // [Hq, total_q], natural log
+  float* part;           // [Hkv, total_q]
+  int32_t total_q, num_q_heads, num_kv_heads, num_pages, log2_group;
+  float scale_log2;      // softmax_scale * log2(e)
+};
+
+struct MassShared {
+  uint64_t item_full[2], item_empty[2];
+  uint64_t k_full, k_empty;
+  uint64_t q_full[4], q_empty[4];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t drain;
+  __align__(16) int32_t item[2][M_NFIELDS];
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D, int P>
+__global__ void __launch_bounds__(192, 1)
+    segpaged_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const MassParams p) {
+  using C = MassCfg<D, P>;
+  static_assert(C::NQ <= 4, "barrier arrays hold four query slots");
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ MassShared sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;                                   // key tile
+  uint8_t* sQ = smem + C::TILE_BYTES;                   // NQ query tiles
+  float* s_nlse = reinterpret_cast<float*>(smem + C::TILE_BYTES * (1 + C::NQ));   // [NQ][128]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort = &sh.abort;
+  int32_t* status = p.status;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&sh.item_full[i], 1);
+      ptx::mbar_init(&sh.item_empty[i], 5);   // MMA warp + 4 mass warps
+      ptx::mbar_init(&sh.s_full[i], 1);
+      ptx::mbar_init(&sh.s_empty[i], 4);
+    }
+    for (int i = 0; i < C::NQ; ++i) {
+      ptx::mbar_init(&sh.q_full[i], 1);
+      ptx::mbar_init(&sh.q_empty[i], 5);      // MMA commit + 4 mass warps (their LSE reads)
+    }
+    ptx::mbar_init(&sh.k_full, 1);
+    ptx::mbar_init(&sh.k_empty, 1);
+    ptx::mbar_init(&sh.drain, 1);
+    sh.abort = 0;
+    ptx::mbar_fence_init();
+  }
+  if (warp == 4 && lane == 0) {
+    ptx::tma_prefetch_desc(&tm_q);
+    ptx::tma_prefetch_desc(&tm_k);
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  // The key tile starts zeroed: pages a tile skips (keys before the query range) keep finite data.
+  for (int x = threadIdx.x; x < C::TILE_BYTES / 16; x += blockDim.x)
+    reinterpret_cast<uint4*>(sK)[x] = make_uint4(0, 0, 0, 0);
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+  const int G = 1 << p.log2_group;
+  const int npos = 128 >> p.log2_group;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------------------ producer
+    uint32_t qi = 0, q_issued = 0;
+    int32_t k_ring = -1;
+    for (uint32_t ring = 0;; ++ring) {
+      const int slot = ring & 1;
+      int go = 1;
+      if (lane == 0) go = ptx::mbar_wait(&sh.item_empty[slot], ((ring >> 1) & 1) ^ 1, abort, status, kMassStatusTimeout);
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      int32_t u = 0;
+      if (lane == 0) u = atomicAdd(p.counter, 1);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      const bool done = u >= p.num_items;
+      int32_t* I = sh.item[slot];
+      if (done) {
+        if (lane == 0) I[M_NT] = -1;
+      } else if (lane < M_NFIELDS / 4) {
+        reinterpret_cast<int4*>(I)[lane] = reinterpret_cast<const int4*>(p.items + (int64_t)u * M_NFIELDS)[lane];
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.item_full[slot]);
+      if (done) break;
+      const int32_t x = I[M_TILE], q0 = I[M_Q0], L = I[M_L], kvh = I[M_KVH], qrow0 = I[M_QROW0];
+      const int32_t t0 = I[M_T0], nt = I[M_NT], Lq = I[M_LQ];
+      // key tile: the pages holding a key of the query range
+      if (lane == 0) {
+        go = ptx::mbar_wait(&sh.k_empty, (ring & 1) ^ 1, abort, status, kMassStatusTimeout);
+        if (go) {
+          int32_t pid[C::PPT];
+          int32_t n_ok = 0;
+#pragma unroll
+          for (int c = 0; c < C::PPT; ++c) {
+            const int32_t lp = x * C::PPT + c;
+            pid[c] = -1;
+            if ((int64_t)lp * P + P <= q0 || (int64_t)lp * P >= L) continue;
+            const int32_t idx = I[M_GLOBAL] ? lp : (lp < I[M_NSINK] ? lp : I[M_NSINK] + (lp - I[M_W0]));
+            if (idx < 0 || idx >= I[M_TOTAL] || (int64_t)I[M_TOFF] + idx >= p.page_table_len) {
+              if (status) atomicOr(status, kMassStatusUnit);
+              continue;
+            }
+            int32_t v = p.page_table[(int64_t)I[M_TOFF] + idx];
+            if (v < 0 || v >= p.num_pages) {
+              if (status) atomicOr(status, kMassStatusPageId);
+              v = 0;
+            }
+            pid[c] = v;
+            ++n_ok;
+          }
+          ptx::mbar_arrive_expect_tx(&sh.k_full, (uint32_t)(n_ok * P * D * 2));
+#pragma unroll
+          for (int c = 0; c < C::PPT; ++c) {
+            if (pid[c] < 0) continue;
+#pragma unroll
+            for (int h = 0; h < C::NH; ++h)
+              ptx::tma_load_3d(sK + h * C::BLK + c * P * 128, &tm_k, h * 64, 0, pid[c], &sh.k_full);
+          }
+          k_ring = (int32_t)ring;
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      // query tiles with their rows' -LSE * log2(e)
+      for (int32_t t = t0; t < t0 + nt; ++t, ++qi) {
+        const int s = qi % C::NQ;
+        if (lane == 0) go = ptx::mbar_wait(&sh.q_empty[s], ((qi / C::NQ) & 1) ^ 1, abort, status, kMassStatusTimeout);
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c = lane + 32 * k;
+          const int32_t posl = t * npos + (c >> p.log2_group);
+          float v = -INFINITY;
+          if (posl < Lq && qrow0 + posl < p.total_q) {
+            const int32_t head = kvh * G + (c & (G - 1));
+            v = -p.lse[(int64_t)head * p.total_q + qrow0 + posl] * 1.4426950408889634f;
+          }
+          s_nlse[s * 128 + c] = v;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&sh.q_full[s], C::TILE_BYTES);
+#pragma unroll
+          for (int h = 0; h < C::NH; ++h)
+            ptx::tma_load_3d(sQ + s * C::TILE_BYTES + h * C::BLK, &tm_q, h * 64, kvh * G, qrow0 + t * npos,
+                             &sh.q_full[s]);
+          q_issued = qi + 1;
+        }
+      }
+      if (!go) break;
+    }
+    // After giving up, wait (bounded, ignoring the abort flag) for this warp's copies in flight.
+    if (lane == 0 && *abort) {
+      if (k_ring >= 0) ptx::mbar_wait(&sh.k_full, (uint32_t)k_ring & 1, nullptr, status, kMassStatusTimeout);
+      const uint32_t first = q_issued > (uint32_t)C::NQ ? q_issued - C::NQ : 0u;
+      for (uint32_t it = first; it < q_issued; ++it)
+        ptx::mbar_wait(&sh.q_full[it % C::NQ], (it / C::NQ) & 1, nullptr, status, kMassStatusTimeout);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // --------------------------------------------------------------------------- MMA issuer
+    const uint32_t leader = ptx::elect_one();
+    const uint32_t k_base = ptx::smem_addr(sK), q_base = ptx::smem_addr(sQ);
+    const uint64_t kdesc = ptx::sw128_desc(k_base, 16, 1024);
+    uint32_t qi = 0, si = 0;
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kMassStatusTimeout));
+    };
+    bool ok = true;
+    for (uint32_t ring = 0; ok; ++ring) {
+      const int slot = ring & 1;
+      if (!wait(&sh.item_full[slot], (ring >> 1) & 1)) break;
+      const int32_t nt = sh.item[slot][M_NT];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.item_empty[slot]);
+      if (nt < 0) break;
+      if (!wait(&sh.k_full, ring & 1)) break;
+      for (int32_t t = 0; t < nt; ++t, ++qi, ++si) {
+        const int s = qi % C::NQ, b = si & 1;
+        if (!wait(&sh.q_full[s], (qi / C::NQ) & 1) || !wait(&sh.s_empty[b], ((si >> 1) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint64_t qdesc = ptx::sw128_desc(q_base + s * C::TILE_BYTES, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * C::BLK + (kk & 3) * 32) >> 4);
+          ptx::umma_ss(leader, tmem + b * 128, kdesc + off, qdesc + off, C::IDESC, kk > 0 ? 1u : 0u);
+        }
+        ptx::umma_commit(leader, &sh.s_full[b]);
+        ptx::umma_commit(leader, &sh.q_empty[s]);
+      }
+      if (!ok) break;
+      ptx::umma_commit(leader, &sh.k_empty);
+    }
+    __syncwarp();
+    ptx::umma_commit(leader, &sh.drain);
+    ptx::mbar_wait(&sh.drain, 0, nullptr, status, kMassStatusTimeout);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------------ mass warpgroup
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;                 // key row of the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint64_t sl2_2 = (uint64_t)__float_as_uint(p.scale_log2) |
+                           ((uint64_t)__float_as_uint(p.scale_log2) << 32);
+    uint32_t qi = 0, si = 0;
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kMassStatusTimeout));
+    };
+    for (uint32_t ring = 0;; ++ring) {
+      const int slot = ring & 1;
+      if (!wwait(&sh.item_full[slot], (ring >> 1) & 1)) break;
+      const int32_t* I = sh.item[slot];
+      const int32_t nt = I[M_NT];
+      if (nt < 0) {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.item_empty[slot]);
+        break;
+      }
+      const int32_t j = I[M_TILE] * 128 + row;           // this thread's key position
+      const int32_t q0 = I[M_Q0], t0 = I[M_T0];
+      const bool is_global = I[M_GLOBAL] != 0;
+      const int32_t S = I[M_SINK], W = I[M_WIN];
+      float sum = 0.f;
+      bool ok = true;
+      for (int32_t t = 0; t < nt; ++t, ++qi, ++si) {
+        const int s = qi % C::NQ, b = si & 1;
+        if (!wwait(&sh.s_full[b], (si >> 1) & 1) || !wwait(&sh.q_full[s], (qi / C::NQ) & 1)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        float v[128];
+        const uint32_t sbuf = tmem + b * 128 + lane_off;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(sbuf + c * 32, reinterpret_cast<uint32_t*>(v) + c * 32);
+        ptx::tmem_ld_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.s_empty[b]);
+        // The query tile's positions [pa, pb]; which of them see key j.
+        const int32_t pa = q0 + (t0 + t) * npos, pb = pa + npos - 1;
+        const bool none = j > pb || (!is_global && j >= S && j <= pa - W);
+        const bool all = j <= pa && (is_global || j < S || j > pb - W);
+        if (!none) {
+          const float* nl = s_nlse + s * 128;
+          uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            const float2 n2 = *reinterpret_cast<const float2*>(nl + c);
+            uint64_t x2;
+            asm("fma.rn.f32x2 %0, %1, %2, %3;"
+                : "=l"(x2)
+                : "l"((uint64_t)__float_as_uint(v[c]) | ((uint64_t)__float_as_uint(v[c + 1]) << 32)), "l"(sl2_2),
+                  "l"((uint64_t)__float_as_uint(n2.x) | ((uint64_t)__float_as_uint(n2.y) << 32)));
+            float x0 = __uint_as_float((uint32_t)x2), x1 = __uint_as_float((uint32_t)(x2 >> 32));
+            if (!all) {
+              const int32_t i0 = pa + (c >> p.log2_group), i1 = pa + ((c + 1) >> p.log2_group);
+              if (!(j <= i0 && (is_global || j < S || j > i0 - W))) x0 = -INFINITY;
+              if (!(j <= i1 && (is_global || j < S || j > i1 - W))) x1 = -INFINITY;
+            }
+            const uint64_t e2 = (uint64_t)__float_as_uint(ptx::ex2(x0)) | ((uint64_t)__float_as_uint(ptx::ex2(x1)) << 32);
+            asm("add.rn.f32x2 %0, %1, %2;" : "=l"(acc[(c >> 1) & 3]) : "l"(acc[(c >> 1) & 3]), "l"(e2));
+          }
+          uint64_t t2;
+          asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(acc[0]), "l"(acc[1]));
+          uint64_t u2;
+          asm("add.rn.f32x2 %0, %1, %2;" : "=l"(u2) : "l"(acc[2]), "l"(acc[3]));
+          asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(t2), "l"(u2));
+          sum += __uint_as_float((uint32_t)t2) + __uint_as_float((uint32_t)(t2 >> 32));
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.q_empty[s]);
+      }
+      if (!ok) break;
+      if (j >= q0 && j < I[M_L]) {
+        const int64_t r = (int64_t)I[M_QROW0] + (j - q0);
+        if (I[M_KVH] >= 0 && I[M_KVH] < p.num_kv_heads && r < p.total_q) p.part[(int64_t)I[M_KVH] * p.total_q + r] = sum;
+        else if (status) atomicOr(status, kMassStatusUnit);
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.item_empty[slot]);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// mass[r] = sum over KV heads k (in order) of part[k][r].
+__global__ void mass_reduce_kernel(const float* __restrict__ part, float* __restrict__ mass, int32_t total_q,
+                                   int32_t num_kv_heads) {
+  for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < total_q; r += (int64_t)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int k = 0; k < num_kv_heads; ++k) s += part[(int64_t)k * total_q + r];
+    mass[r] = s;
+  }
+}
+
+}  // namespace segpaged

@@ -37,6 +37,9 @@ class LayerState:
     lse: torch.Tensor | None = None
     stored_bytes: int = 0
     dense_bytes: int = 0
+    mass_items: np.ndarray | None = None     # token-mass plan (sparse-FFN score)
+    mass_items_dev: torch.Tensor | None = None
+    mass: torch.Tensor | None = None
 
 
 class Runner:
@@ -45,10 +48,11 @@ class Runner:
     shared_dense: all layers scatter the same dense K/V (drawn for layer 0) through their own tables,
     class maps and queries -- for many-layer workloads whose dense K/V would not fit in memory at once.
     keep_dense: keep each layer's dense K/V on the device after set-up (tests compare against them).
+    mass: also plan and hold the per-token attention mass (the sparse-FFN score) of every layer.
     """
 
     def __init__(self, w: synth.Workload, device="cuda", layers=None, keep_dense=False, page_seed_offset=0,
-                 shared_dense=False, split_ctas=None):
+                 shared_dense=False, split_ctas=None, mass=False):
         self.w = w
         self.device = torch.device(device)
         # long units are split across CTAs when one alone exceeds a CTA's share (short query ranges)
@@ -84,6 +88,9 @@ class Runner:
         self.ql_dev = torch.from_numpy(self.ql).to(self.device)
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.workspace = None
+        self.mass_workspace = None
+        self.with_mass = mass
+        self.cu_q_dev = torch.from_numpy(w.cu_q().astype(np.int32)).to(self.device)
         self.rope = None
         if w.rope_theta is not None:
             self.rope = torch.from_numpy(sp.segpaged_rope_cos_sin(w.rope_theta, w.rope_deltas, D)).to(self.device)
@@ -119,6 +126,13 @@ class Runner:
         need = sp.segpaged_prefill_workspace_bytes(self.dims, st.info)
         if self.workspace is None or self.workspace.numel() * 4 < need:
             self.workspace = torch.zeros((need + 3) // 4, dtype=torch.int32, device=self.device)
+        if self.with_mass:
+            self.plan_mass(li)
+            st.mass_items_dev = torch.from_numpy(np.ascontiguousarray(st.mass_items)).to(self.device)
+            st.mass = torch.zeros(w.total_q, dtype=torch.float32, device=self.device)
+            need = sp.segpaged_mass_workspace_bytes(self.dims, w.total_q)
+            if self.mass_workspace is None or self.mass_workspace.numel() * 4 < need:
+                self.mass_workspace = torch.zeros((need + 3) // 4, dtype=torch.int32, device=self.device)
 
     def dense_of(self, li):
         if self._tmp_dense is not None:
@@ -161,6 +175,22 @@ class Runner:
         st = self.state[li]
         sp.segpaged_attn_prefill(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info,
                                  self.scale, st.o, st.lse, self.workspace, self.status, stream)
+
+    def plan_mass(self, li):
+        """Host planning of one layer's token-mass items."""
+        st = self.state[li]
+        st.mass_items = sp.segpaged_mass_plan(self.dims, self.ctx, self.ql, st.cls, st.offs)
+        return st.mass_items
+
+    def token_mass(self, li, stream=None):
+        """Attention mass each query row's token receives (needs this layer's prefill LSE)."""
+        st = self.state[li]
+        sp.segpaged_token_mass(self.dims, st.q, self.k_pool, st.table_dev, st.mass_items_dev, st.lse, self.scale, st.mass,
+                               self.mass_workspace, self.status, stream)
+
+    def select_topk(self, li, k_per_seq: torch.Tensor, selected: torch.Tensor, stream=None):
+        """Top-k rows per sequence by this layer's mass into `selected`."""
+        sp.segpaged_select_topk(self.state[li].mass, self.cu_q_dev, k_per_seq, selected, stream)
 
     def step(self, stream=None):
         """Prefill of every layer (pools and plans already in place)."""

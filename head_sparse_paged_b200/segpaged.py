@@ -16,6 +16,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsegpaged.so")
 UNIT_FIELDS = 32
+MASS_ITEM_FIELDS = 16
 
 STATUS_PAGE_ID = 1
 STATUS_TABLE = 2
@@ -25,7 +26,8 @@ STATUS_UNIT = 8
 # Every function include/segpaged.h declares.
 EXPORTS = ("segpaged_error_string", "segpaged_pages_bytes", "segpaged_rope_cos_sin", "segpaged_build",
            "segpaged_prefill_plan", "segpaged_prefill_workspace_bytes", "segpaged_attn_prefill",
-           "segpaged_attn_prefill_noalloc")
+           "segpaged_attn_prefill_noalloc", "segpaged_mass_plan", "segpaged_mass_workspace_bytes",
+           "segpaged_token_mass", "segpaged_select_topk")
 
 
 class SegPagedError(RuntimeError):
@@ -80,6 +82,15 @@ def _load():
                                           ctypes.c_size_t, vp, vp]
     lib.segpaged_attn_prefill_noalloc.restype = ctypes.c_int
     lib.segpaged_attn_prefill_noalloc.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, i64, ctypes.c_float, vp, vp, vp, vp]
+    lib.segpaged_mass_plan.restype = i64
+    lib.segpaged_mass_plan.argtypes = [dp, vp, vp, vp, vp, vp, i64]
+    lib.segpaged_mass_workspace_bytes.restype = ctypes.c_size_t
+    lib.segpaged_mass_workspace_bytes.argtypes = [dp, i32]
+    lib.segpaged_token_mass.restype = ctypes.c_int
+    lib.segpaged_token_mass.argtypes = [dp, vp, i32, vp, vp, i64, vp, i64, vp, ctypes.c_float, vp, vp, ctypes.c_size_t,
+                                        vp, vp]
+    lib.segpaged_select_topk.restype = ctypes.c_int
+    lib.segpaged_select_topk.argtypes = [i32, vp, vp, vp, vp, vp]
     return lib
 
 
@@ -224,3 +235,48 @@ def segpaged_attn_prefill_noalloc(dims: Dims, q, k_pool, v_pool, page_table, uni
                                            _stream(stream))
     if r < 0:
         raise SegPagedError(r, "segpaged_attn_prefill_noalloc")
+
+
+def segpaged_mass_plan(dims: Dims, ctx_len, q_len, cls, page_table_offs) -> np.ndarray:
+    """Work items (int32 [n, 16]) of segpaged_token_mass, longest first. Host only."""
+    B, H = dims.num_seqs, dims.num_kv_heads
+    L, Lq = _host_i32(ctx_len, B), _host_i32(q_len, B)
+    c, offs = _host_i32(cls, B * H * 3), _host_i32(page_table_offs, B * H + 1)
+    d = dims.c()
+    n = _lib.segpaged_mass_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), None, 0)
+    if n < 0:
+        raise SegPagedError(int(n), "segpaged_mass_plan")
+    items = np.zeros((max(n, 1), MASS_ITEM_FIELDS), np.int32)
+    n2 = _lib.segpaged_mass_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), _hp(items), n)
+    if n2 < 0:
+        raise SegPagedError(int(n2), "segpaged_mass_plan")
+    return items[:n]
+
+
+def segpaged_mass_workspace_bytes(dims: Dims, total_q: int) -> int:
+    return int(_lib.segpaged_mass_workspace_bytes(ctypes.byref(dims.c()), int(total_q)))
+
+
+def segpaged_token_mass(dims: Dims, q, k_pool, page_table, items, lse, softmax_scale, mass, workspace, status=None,
+                        stream=None):
+    """mass [total_q] float32 (CUDA), written in place: the attention mass each query row's token receives.
+    items: the mass plan on the device; lse: the prefill's LSE [Hq, total_q] for the same inputs."""
+    bf = torch.bfloat16
+    r = _lib.segpaged_token_mass(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]), _dev(k_pool, bf, "k_pool"),
+                                 _dev(page_table, torch.int32, "page_table"), int(page_table.numel()),
+                                 _dev(items, torch.int32, "items"), int(items.shape[0]), _dev(lse, torch.float32, "lse"),
+                                 float(softmax_scale), _dev(mass, torch.float32, "mass"),
+                                 _dev(workspace, None, "workspace"), int(workspace.numel() * workspace.element_size()),
+                                 _dev(status, torch.int32, "status"), _stream(stream))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_token_mass")
+
+
+def segpaged_select_topk(mass, cu_seqlens_q, k_per_seq, selected, stream=None):
+    """Top-k rows per sequence by mass into `selected` (int32, CUDA), ascending within each sequence."""
+    r = _lib.segpaged_select_topk(int(cu_seqlens_q.numel()) - 1, _dev(mass, torch.float32, "mass"),
+                                  _dev(cu_seqlens_q, torch.int32, "cu_seqlens_q"),
+                                  _dev(k_per_seq, torch.int32, "k_per_seq"), _dev(selected, torch.int32, "selected"),
+                                  _stream(stream))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_select_topk")

@@ -234,3 +234,63 @@ def test_validation_errors():
                                      None, None, None, 256, None, None) == -1
     assert lib.segpaged_build(ctypes.byref(dims.c()), *([None] * 12)) == -1
     assert sp.error_string(-5).startswith("page-table")
+
+
+# Mass item field positions (head_sparse_paged_b200/csrc/mass_sm100.cuh).
+(M_SEQ, M_KVH, M_TILE, M_TOFF, M_NSINK, M_W0, M_GLOBAL, M_SINK, M_WIN, M_Q0, M_L, M_QROW0, M_T0, M_NT, M_TOTAL,
+ M_LQ) = range(16)
+
+
+@pytest.mark.parametrize("case", range(len(EDGE)))
+def test_mass_plan_covers_every_query_key_and_every_viewer(case):
+    """Each (sequence, KV head) gets one item per 128-key tile that holds a key of the query range;
+    an item's query tiles [t0, t0 + nt) include every query tile with a row that sees one of those
+    keys (the oracle's visibility rule) and start and end on such tiles; the key pages it reads are
+    stored, at the table index the storage order gives; items come longest first."""
+    w_seqs, Hq, Hkv, D, P, classes = EDGE[case]
+    B = len(w_seqs)
+    dims = sp.Dims(B, Hq, Hkv, D, P)
+    ctx = [s[0] for s in w_seqs]
+    ql = [s[1] for s in w_seqs]
+    cls = np.asarray(classes, np.int32)
+    _, _, per = sp.segpaged_pages_bytes(dims, ctx, ql, cls)
+    offs = np.concatenate([[0], np.cumsum(per)]).astype(np.int32)
+    items = sp.segpaged_mass_plan(dims, ctx, ql, cls, offs)
+    G = Hq // Hkv
+    npos = 128 // G
+    cu_q = np.concatenate([[0], np.cumsum(ql)])
+    nts = [int(it[M_NT]) for it in items]
+    assert nts == sorted(nts, reverse=True)
+    got = {}
+    for it in items:
+        b, kh, x = int(it[M_SEQ]), int(it[M_KVH]), int(it[M_TILE])
+        assert (b, kh, x) not in got
+        got[(b, kh, x)] = it
+        L, Lq = ctx[b], ql[b]
+        q0 = L - Lq
+        g, S, W = (int(v) for v in cls[b, kh])
+        assert (it[M_Q0], it[M_L], it[M_LQ], it[M_QROW0]) == (q0, L, Lq, cu_q[b])
+        assert it[M_TOFF] == offs[b * Hkv + kh]
+        stored = orc.stored_logical_pages(L, Lq, bool(g), S, W, P)
+        assert it[M_TOTAL] == len(stored)
+        for c in range(128 // P):            # pages with a key of the query range are stored, at their index
+            lp = x * (128 // P) + c
+            if lp * P + P <= q0 or lp * P >= L:
+                continue
+            idx = lp if g else (lp if lp < it[M_NSINK] else int(it[M_NSINK]) + lp - int(it[M_W0]))
+            assert stored[idx] == lp
+        viewers = set()
+        jmin, jmax = max(q0, 128 * x), min(L, 128 * x + 128) - 1
+        for i in range(q0, L):
+            v = orc.visible_keys(bool(g), S, W, i)
+            at = int(np.searchsorted(v, jmin))
+            if at < len(v) and v[at] <= jmax:
+                viewers.add((i - q0) // npos)
+        t0, nt = int(it[M_T0]), int(it[M_NT])
+        assert viewers <= set(range(t0, t0 + nt))
+        assert t0 in viewers and t0 + nt - 1 in viewers
+    for b in range(B):
+        L, Lq = ctx[b], ql[b]
+        for kh in range(Hkv):
+            want = set(range((L - Lq) // 128, (L - 1) // 128 + 1)) if Lq > 0 else set()
+            assert {x for (bb, k, x) in got if bb == b and k == kh} == want
