@@ -47,6 +47,10 @@ def parse_args(argv=None):
                     help="ours: the SegPaged library; reference: the fp64 oracle on the host cores; dense: "
                          "the dense-layout baseline (PyTorch SDPA, all heads at full context, explicit mask)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-mass", action="store_true",
+                    help="skip the token-mass / top-k selection measurement (sparse-FFN score)")
+    ap.add_argument("--topk-frac", type=float, default=0.25,
+                    help="share of each sequence's query tokens the top-k selection keeps")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle sample")
     return ap.parse_args(argv)
@@ -378,7 +382,7 @@ def run_ours(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = rank_workload(args.workload, rank)
-    runner = Runner(w, device=device, keep_dense=True, shared_dense=(w.layers > 1))
+    runner = Runner(w, device=device, keep_dense=True, shared_dense=(w.layers > 1), mass=not args.no_mass)
     torch.cuda.synchronize()
     runner.check_status()
     flops_layer = {li: visible_flops(w, [li]) for li in runner.layers}
@@ -450,6 +454,9 @@ def run_ours(args, rank, world, local):
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(runner, args, world, device, flops_step)
+    mass = None
+    if not args.no_mass:
+        mass = measure_mass(runner, args, world, device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -481,11 +488,76 @@ def run_ours(args, rank, world, local):
                      "peak_source": f"{src} {peak_name}", "kernel": "segpaged_prefill_kernel"},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "token_mass": mass,
         "gpu_launches": args.steps * n_layers * 2,
         "clocks": clocks,
     }
     print(json.dumps(line))
     return 0
+
+
+# MUFU peak for the token-mass pass: 16 ex2 per clock per SM (sm_100), 148 SMs, at the maximum SM clock.
+MUFU_EX2_PER_CLK_SM = 16
+
+
+def mass_pairs(w, layer):
+    """Visible (query row, query head, key of the query range) triples of one layer: one exp2 each."""
+    import numpy as np
+    total = 0
+    for b in range(w.num_seqs):
+        L, Lq = w.ctx_lens[b], w.q_lens[b]
+        j = np.arange(L - Lq, L, dtype=np.int64)
+        for kh in range(w.num_kv_heads):
+            g, S, W = (int(x) for x in w.classes[layer, b, kh])
+            n = (L - j) if g else np.where(j < S, L - j, np.minimum(L - j, W))
+            total += w.group * int(n.sum())
+    return total
+
+
+def measure_mass(runner, args, world, device):
+    """Token-mass pass plus top-k selection of every layer, after the timed prefill steps (it needs their
+    LSE): CUDA events around each mass launch, K steps after W warm-up steps."""
+    import numpy as np
+    import torch
+    w = runner.w
+    stream = torch.cuda.current_stream()
+    k_per_seq = torch.tensor([max(1, int(round(args.topk_frac * l))) for l in w.q_lens], dtype=torch.int32,
+                             device=device)
+    selected = torch.empty(int(k_per_seq.sum().item()), dtype=torch.int32, device=device)
+    pairs = {li: mass_pairs(w, li) for li in runner.layers}
+    for _ in range(args.warmup):
+        for li in runner.layers:
+            runner.token_mass(li)
+            runner.select_topk(li, k_per_seq, selected)
+    torch.cuda.synchronize()
+    ev = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        for li in runner.layers:
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            runner.token_mass(li)
+            b.record(stream)
+            runner.select_topk(li, k_per_seq, selected)
+            ev.append((li, a, b))
+    t1.record(stream)
+    torch.cuda.synchronize()
+    runner.check_status()
+    total_ms = t0.elapsed_time(t1)
+    mass_ms = sum(a.elapsed_time(b) for _, a, b in ev)
+    exps = sum(pairs[li] for li, _, _ in ev)
+    peaks, _ = load_peaks()
+    clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    peak = MUFU_EX2_PER_CLK_SM * torch.cuda.get_device_properties(device).multi_processor_count * clk
+    achieved = exps / (mass_ms * 1e-3)
+    return {"kernel": "segpaged_mass_kernel (+ reduce)", "ms_per_layer": mass_ms / len(ev),
+            "with_topk_ms_per_layer": total_ms / len(ev), "visible_pairs_per_step": sum(pairs.values()),
+            "bound": "alu", "achieved": achieved / 1e9, "peak": peak / 1e9, "unit": "G exp2/s",
+            "frac": achieved / peak, "peak_source": f"{MUFU_EX2_PER_CLK_SM} ex2/clk/SM x SMs x sm_max_mhz",
+            "topk_frac": args.topk_frac}
 
 
 def measure_e2e(runner, args, world, device, flops_step):

@@ -11,15 +11,17 @@
 // it. Logits are computed transposed, S^T = K Q^T (tcgen05.mma, M = 128 keys, N = 128 query rows,
 // both operands K-major in 128B-swizzled shared memory, f32 in TMEM), so each thread of the mass
 // warpgroup owns one key's TMEM lane and sums its row: no cross-thread reduction. The sum of an item
-// goes to a per-(KV head, query row) partial; mass_reduce_kernel adds the KV heads in a fixed order.
+// goes to a per-(warpgroup, KV head, query row) partial; mass_reduce_kernel adds them in a fixed order.
 //
-// Per CTA, 6 warps:
-//   warps 0-3  mass: tcgen05.ld of the key's 128 logits, exp2(s * scale * log2 e - LSE_i * log2 e) with
-//              per-element bounds only on edge pairs, running sum in packed f32x2.
-//   warp 4     producer: claims items, TMA-loads the key tile's pages once and every query tile
+// Per CTA, 10 warps:
+//   warps 0-3, 4-7  two mass warpgroups, taking the item's query tiles alternately (tile parity picks
+//              the warpgroup and its TMEM buffer), so one exponentiates while the other waits on its
+//              logits: tcgen05.ld of the key's 128 logits, exp2(s * scale * log2 e - LSE_i * log2 e)
+//              with per-element bounds only on edge pairs, running sum in packed f32x2.
+//   warp 8     producer: claims items, TMA-loads the key tile's pages once and every query tile
 //              (same map as the prefill), and gathers the 128 rows' -LSE * log2 e into shared memory
 //              (+inf LSE for rows past the query range, so they contribute exp2(-inf) = 0).
-//   warp 5     MMA issuer (whole warp, one elected lane issues): S^T into one of two TMEM buffers.
+//   warp 9     MMA issuer (whole warp, one elected lane issues): S^T into one of two TMEM buffers.
 // Every wait is bounded, as in the prefill kernel.
 #pragma once
 #include <cuda.h>
@@ -61,10 +63,10 @@ struct MassCfg {
   static constexpr int NH = D / 64;                   // 128-byte swizzle column blocks across D
   static constexpr int BLK = 128 * 128;               // bytes of one 64-column block of a 128-row tile
   static constexpr int TILE_BYTES = 128 * D * 2;      // key tile or query tile
-  static constexpr int NQ = 3;                        // query-tile ring
+  static constexpr int NQ = 4;                        // query-tile ring
   static constexpr int PPT = 128 / P;                 // pages per key tile
   static constexpr int SMEM_BYTES = TILE_BYTES * (1 + NQ) + NQ * 128 * 4 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 256;          // two S^T buffers of 128 columns
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, 128, 0, 0);
 };
@@ -77,7 +79,7 @@ struct MassParams {
   int32_t* counter;      // zeroed before the launch
   int32_t* status;       // nullable
   const float* lse;      // [Hq, total_q], natural log
-  float* part;           // [Hkv, total_q]
+  float* part;           // [2 warpgroups][Hkv][total_q]
   int32_t total_q, num_q_heads, num_kv_heads, num_pages, log2_group;
   float scale_log2;      // softmax_scale * log2(e)
 };
@@ -94,7 +96,7 @@ struct MassShared {
 };
 
 template <int D, int P>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     segpaged_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const MassParams p) {
   using C = MassCfg<D, P>;
@@ -112,13 +114,13 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sh.item_full[i], 1);
-      ptx::mbar_init(&sh.item_empty[i], 5);   // MMA warp + 4 mass warps
+      ptx::mbar_init(&sh.item_empty[i], 9);   // MMA warp + 8 mass warps
       ptx::mbar_init(&sh.s_full[i], 1);
-      ptx::mbar_init(&sh.s_empty[i], 4);
+      ptx::mbar_init(&sh.s_empty[i], 4);      // the 4 warps of the buffer's warpgroup
     }
     for (int i = 0; i < C::NQ; ++i) {
       ptx::mbar_init(&sh.q_full[i], 1);
-      ptx::mbar_init(&sh.q_empty[i], 5);      // MMA commit + 4 mass warps (their LSE reads)
+      ptx::mbar_init(&sh.q_empty[i], 5);      // MMA commit + the 4 warps that read the tile's LSE
     }
     ptx::mbar_init(&sh.k_full, 1);
     ptx::mbar_init(&sh.k_empty, 1);
@@ -126,11 +128,11 @@ __global__ void __launch_bounds__(192, 1)
     sh.abort = 0;
     ptx::mbar_fence_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     ptx::tma_prefetch_desc(&tm_q);
     ptx::tma_prefetch_desc(&tm_k);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(192, 1)
   const int G = 1 << p.log2_group;
   const int npos = 128 >> p.log2_group;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------------------------ producer
     uint32_t qi = 0, q_issued = 0;
     int32_t k_ring = -1;
@@ -205,21 +207,32 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
-      // query tiles with their rows' -LSE * log2(e)
-      for (int32_t t = t0; t < t0 + nt; ++t, ++qi) {
-        const int s = qi % C::NQ;
-        if (lane == 0) go = ptx::mbar_wait(&sh.q_empty[s], ((qi / C::NQ) & 1) ^ 1, abort, status, kMassStatusTimeout);
-        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      // query tiles with their rows' -LSE * log2(e); the values of the next tile are loaded while the
+      // current one waits for its slot and is issued, so the gather's latency stays off the critical path
+      auto gather = [&](int32_t t, float (&nl)[4]) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int c = lane + 32 * k;
           const int32_t posl = t * npos + (c >> p.log2_group);
-          float v = -INFINITY;
+          nl[k] = -INFINITY;
           if (posl < Lq && qrow0 + posl < p.total_q) {
             const int32_t head = kvh * G + (c & (G - 1));
-            v = -p.lse[(int64_t)head * p.total_q + qrow0 + posl] * 1.4426950408889634f;
+            nl[k] = -p.lse[(int64_t)head * p.total_q + qrow0 + posl] * 1.4426950408889634f;
           }
-          s_nlse[s * 128 + c] = v;
+        }
+      };
+      float cur[4];
+      gather(t0, cur);
+      for (int32_t t = t0; t < t0 + nt; ++t, ++qi) {
+        const int s = qi % C::NQ;
+        float nxt[4] = {0.f, 0.f, 0.f, 0.f};
+        if (t + 1 < t0 + nt) gather(t + 1, nxt);
+        if (lane == 0) go = ptx::mbar_wait(&sh.q_empty[s], ((qi / C::NQ) & 1) ^ 1, abort, status, kMassStatusTimeout);
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          s_nlse[s * 128 + lane + 32 * k] = cur[k];
+          cur[k] = nxt[k];
         }
         __syncwarp();
         if (lane == 0) {
@@ -241,7 +254,7 @@ __global__ void __launch_bounds__(192, 1)
         ptx::mbar_wait(&sh.q_full[it % C::NQ], (it / C::NQ) & 1, nullptr, status, kMassStatusTimeout);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // --------------------------------------------------------------------------- MMA issuer
     const uint32_t leader = ptx::elect_one();
     const uint32_t k_base = ptx::smem_addr(sK), q_base = ptx::smem_addr(sQ);
@@ -283,12 +296,12 @@ __global__ void __launch_bounds__(192, 1)
     ptx::mbar_wait(&sh.drain, 0, nullptr, status, kMassStatusTimeout);
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------------ mass warpgroup
+    // ----------------------------------------------------------------------- mass warpgroups
+    const int wg = warp >> 2;                            // takes the tiles g with g % 2 == wg
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;                 // key row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint64_t sl2_2 = (uint64_t)__float_as_uint(p.scale_log2) |
-                           ((uint64_t)__float_as_uint(p.scale_log2) << 32);
+    const uint64_t sl2_2 = f2_pack(p.scale_log2, p.scale_log2);
     uint32_t qi = 0, si = 0;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kMassStatusTimeout));
@@ -311,49 +324,58 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       for (int32_t t = 0; t < nt; ++t, ++qi, ++si) {
         const int s = qi % C::NQ, b = si & 1;
+        if (b != wg) continue;
         if (!wwait(&sh.s_full[b], (si >> 1) & 1) || !wwait(&sh.q_full[s], (qi / C::NQ) & 1)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        float v[128];
-        const uint32_t sbuf = tmem + b * 128 + lane_off;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(sbuf + c * 32, reinterpret_cast<uint32_t*>(v) + c * 32);
-        ptx::tmem_ld_wait();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.s_empty[b]);
         // The query tile's positions [pa, pb]; which of them see key j.
         const int32_t pa = q0 + (t0 + t) * npos, pb = pa + npos - 1;
         const bool none = j > pb || (!is_global && j >= S && j <= pa - W);
         const bool all = j <= pa && (is_global || j < S || j > pb - W);
-        if (!none) {
-          const float* nl = s_nlse + s * 128;
-          uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            const float2 n2 = *reinterpret_cast<const float2*>(nl + c);
-            uint64_t x2;
-            asm("fma.rn.f32x2 %0, %1, %2, %3;"
-                : "=l"(x2)
-                : "l"((uint64_t)__float_as_uint(v[c]) | ((uint64_t)__float_as_uint(v[c + 1]) << 32)), "l"(sl2_2),
-                  "l"((uint64_t)__float_as_uint(n2.x) | ((uint64_t)__float_as_uint(n2.y) << 32)));
-            float x0 = __uint_as_float((uint32_t)x2), x1 = __uint_as_float((uint32_t)(x2 >> 32));
-            if (!all) {
-              const int32_t i0 = pa + (c >> p.log2_group), i1 = pa + ((c + 1) >> p.log2_group);
-              if (!(j <= i0 && (is_global || j < S || j > i0 - W))) x0 = -INFINITY;
-              if (!(j <= i1 && (is_global || j < S || j > i1 - W))) x1 = -INFINITY;
-            }
-            const uint64_t e2 = (uint64_t)__float_as_uint(ptx::ex2(x0)) | ((uint64_t)__float_as_uint(ptx::ex2(x1)) << 32);
-            asm("add.rn.f32x2 %0, %1, %2;" : "=l"(acc[(c >> 1) & 3]) : "l"(acc[(c >> 1) & 3]), "l"(e2));
+        const float* nl = s_nlse + s * 128;
+        const uint32_t sbuf = tmem + b * 128 + lane_off;
+        uint64_t acc[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        // the key's 128 logits in two halves of 64 columns (fewer live registers); the buffer is released
+        // once the second half is in registers
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float v[64];
+          ptx::tmem_ld32(sbuf + half * 64, reinterpret_cast<uint32_t*>(v));
+          ptx::tmem_ld32(sbuf + half * 64 + 32, reinterpret_cast<uint32_t*>(v) + 32);
+          ptx::tmem_ld_wait();
+          if (half == 1) {
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sh.s_empty[b]);
           }
-          uint64_t t2;
-          asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(acc[0]), "l"(acc[1]));
-          uint64_t u2;
-          asm("add.rn.f32x2 %0, %1, %2;" : "=l"(u2) : "l"(acc[2]), "l"(acc[3]));
-          asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(t2), "l"(u2));
-          sum += __uint_as_float((uint32_t)t2) + __uint_as_float((uint32_t)(t2 >> 32));
+          if (none) continue;
+          if (!all) {
+            // edge pair: logits of rows that cannot see key j drop out (masked before the exponentials,
+            // so the exponential loop below has no per-element branch)
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              const int32_t i = pa + ((half * 64 + c) >> p.log2_group);
+              if (!(j <= i && (is_global || j < S || j > i - W))) v[c] = -INFINITY;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const float4 n4 = *reinterpret_cast<const float4*>(nl + half * 64 + c);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int e = c + 2 * h;
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(v[e], v[e + 1]), sl2_2, h ? f2_pack(n4.z, n4.w) : f2_pack(n4.x, n4.y)), x0, x1);
+              acc[(e >> 1) & 3] = f2_add(acc[(e >> 1) & 3], f2_pack(ptx::ex2(x0), ptx::ex2(x1)));
+            }
+          }
+        }
+        if (!none) {
+          float t0f, t1f;
+          f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), t0f, t1f);
+          sum += t0f + t1f;
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.q_empty[s]);
@@ -361,7 +383,8 @@ __global__ void __launch_bounds__(192, 1)
       if (!ok) break;
       if (j >= q0 && j < I[M_L]) {
         const int64_t r = (int64_t)I[M_QROW0] + (j - q0);
-        if (I[M_KVH] >= 0 && I[M_KVH] < p.num_kv_heads && r < p.total_q) p.part[(int64_t)I[M_KVH] * p.total_q + r] = sum;
+        if (I[M_KVH] >= 0 && I[M_KVH] < p.num_kv_heads && r < p.total_q)
+          p.part[((int64_t)wg * p.num_kv_heads + I[M_KVH]) * p.total_q + r] = sum;
         else if (status) atomicOr(status, kMassStatusUnit);
       }
       __syncwarp();
@@ -371,18 +394,18 @@ __global__ void __launch_bounds__(192, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-// mass[r] = sum over KV heads k (in order) of part[k][r].
+// mass[r] = sum over planes k (warpgroup-major, then KV head, in order) of part[k][r].
 __global__ void mass_reduce_kernel(const float* __restrict__ part, float* __restrict__ mass, int32_t total_q,
-                                   int32_t num_kv_heads) {
+                                   int32_t num_planes) {
   for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < total_q; r += (int64_t)gridDim.x * blockDim.x) {
     float s = 0.f;
-    for (int k = 0; k < num_kv_heads; ++k) s += part[(int64_t)k * total_q + r];
+    for (int k = 0; k < num_planes; ++k) s += part[(int64_t)k * total_q + r];
     mass[r] = s;
   }
 }
