@@ -21,6 +21,10 @@ Everything here is written from the method's definition, in fp64 where it is flo
   ("RoPE位置对齐", shshi.cn, "RedKnot技术原理" 2 "位置无关缓存复用").
 * ``rope_cos_sin`` / ``rope_rotate_bf16`` -- the RoPE delta rotation, rotate-half pairing
   (d, d + D/2), with the bit-exact fp32 rule stated in their docstrings.
+* ``rope_fragment_of`` / ``rope_fragment_keys`` -- the same re-alignment applied per fragment of a
+  sequence (reused document fragments sitting at other offsets than the ones their keys were
+  computed at: shshi.cn, "RedKnot技术原理" 2 "位置无关缓存复用"). Reading: a token belongs to the
+  last fragment that starts at or before it; tokens before the first fragment keep their keys.
 * ``token_mass`` / ``select_topk`` -- the token score of the sparse-FFN selection (top-k tokens by
   attention score run the dense FFN, the rest take the residual path: shshi.cn, "RedKnot技术原理" 3
   "稀疏FFN动态调度"). The pages define neither the score nor ties; the reading used here: a token's
@@ -229,6 +233,31 @@ def rope_rotate_bf16(x: np.ndarray, cs: np.ndarray) -> np.ndarray:
         y1 = np.float32(x1 * c) - np.float32(x2 * s)
         y2 = np.float32(x2 * c) + np.float32(x1 * s)
     return bf16_round(np.concatenate([y1, y2], axis=-1).astype(np.float32))
+
+
+def rope_fragment_of(starts, tok: int) -> int:
+    """Index of the last fragment starting at or before token ``tok`` (starts ascending), or -1."""
+    f = -1
+    for i, s0 in enumerate(starts):
+        if s0 <= tok:
+            f = i
+    return f
+
+
+def rope_fragment_keys(k: np.ndarray, cu_k, frag_offs, frag_start, frag_cs) -> np.ndarray:
+    """Dense keys [total_k, Hkv, D] (bf16 values) after per-fragment re-alignment: token j of sequence b
+    is rotated with the (cos, sin) table frag_cs[f] [D/2, 2] of its fragment f, every KV head alike, by
+    ``rope_rotate_bf16``; tokens before the sequence's first fragment are unchanged."""
+    out = np.array(k, dtype=np.float32, copy=True)
+    for b in range(len(cu_k) - 1):
+        lo, hi = int(frag_offs[b]), int(frag_offs[b + 1])
+        starts = [int(x) for x in frag_start[lo:hi]]
+        for j in range(int(cu_k[b + 1] - cu_k[b])):
+            f = rope_fragment_of(starts, j)
+            if f >= 0:
+                row = int(cu_k[b]) + j
+                out[row] = rope_rotate_bf16(k[row], frag_cs[lo + f])
+    return out
 
 
 def rope_rotate_f64(x: np.ndarray, angle_per_dim: np.ndarray) -> np.ndarray:
