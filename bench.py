@@ -49,6 +49,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-mass", action="store_true",
                     help="skip the token-mass / top-k selection measurement (sparse-FFN score)")
+    ap.add_argument("--no-rope-gather", action="store_true",
+                    help="skip the gather-time RoPE measurement (prefill with per-fragment key re-alignment)")
+    ap.add_argument("--fragment-tokens", type=int, default=4096,
+                    help="tokens per reused fragment in the gather-time RoPE measurement")
     ap.add_argument("--topk-frac", type=float, default=0.25,
                     help="share of each sequence's query tokens the top-k selection keeps")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
@@ -457,6 +461,9 @@ def run_ours(args, rank, world, local):
     mass = None
     if not args.no_mass:
         mass = measure_mass(runner, args, world, device)
+    rope_gather = None
+    if not args.no_rope_gather and runner.rope is None:
+        rope_gather = measure_rope_gather(runner, args, device, flops_layer, prefill_total_ms / args.steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -489,6 +496,7 @@ def run_ours(args, rank, world, local):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "token_mass": mass,
+        "rope_gather": rope_gather,
         "gpu_launches": args.steps * n_layers * 2,
         "clocks": clocks,
     }
@@ -558,6 +566,52 @@ def measure_mass(runner, args, world, device):
             "bound": "alu", "achieved": achieved / 1e9, "peak": peak / 1e9, "unit": "G exp2/s",
             "frac": achieved / peak, "peak_source": f"{MUFU_EX2_PER_CLK_SM} ex2/clk/SM x SMs x sm_max_mhz",
             "topk_frac": args.topk_frac}
+
+
+def measure_rope_gather(runner, args, device, flops_layer, plain_prefill_ms_per_step):
+    """Prefill of every layer with gather-time RoPE: each sequence is a run of reused fragments of
+    --fragment-tokens tokens, each re-aligned from a seeded original offset to where it now sits. Timed like
+    the main prefill launches (CUDA events around each launch), K steps after W warm-up steps."""
+    import numpy as np
+    import torch
+    from head_sparse_paged_b200 import segpaged as sp
+    w = runner.w
+    rng = np.random.default_rng(w.seed + 4242)
+    offs, starts, deltas = [0], [], []
+    for L in w.ctx_lens:
+        st = list(range(0, L, args.fragment_tokens))
+        starts += st
+        deltas += [int(s0 - o) for s0, o in zip(st, rng.integers(0, 1 << 16, size=len(st)))]
+        offs.append(len(starts))
+    tab = sp.segpaged_rope_cos_sin(1e6, deltas, w.head_dim)
+    runner.frags = (torch.tensor(offs, dtype=torch.int32, device=device),
+                    torch.tensor(starts, dtype=torch.int32, device=device),
+                    torch.from_numpy(tab).to(device))
+    stream = torch.cuda.current_stream()
+    try:
+        for _ in range(args.warmup):
+            for li in runner.layers:
+                runner.prefill(li)
+        torch.cuda.synchronize()
+        ev = []
+        for _ in range(args.steps):
+            for li in runner.layers:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                runner.prefill(li)
+                b.record(stream)
+                ev.append((li, a, b))
+        torch.cuda.synchronize()
+        runner.check_status()
+    finally:
+        runner.frags = None
+    ms = sum(a.elapsed_time(b) for _, a, b in ev)
+    flops = sum(flops_layer[li] for li, _, _ in ev)
+    per_step = ms / args.steps
+    return {"kernel": "segpaged_prefill_kernel<ROPE>", "fragment_tokens": args.fragment_tokens,
+            "fragments": len(starts), "prefill_ms_per_layer": ms / len(ev),
+            "tflops": flops / (ms * 1e-3) / 1e12, "time_vs_plain_prefill": per_step / plain_prefill_ms_per_step}
 
 
 def measure_e2e(runner, args, world, device, flops_step):

@@ -8,7 +8,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsegpaged.so")
 SOURCES = ["segpaged_api.cu", "segpaged_mass.cu"]
-HEADERS = ["sm100_ptx.cuh", "plan.h", "host_common.h", "build_kernel.cuh", "prefill_sm100.cuh", "combine_kernel.cuh",
+HEADERS = ["sm100_ptx.cuh", "plan.h", "host_common.h", "rope.cuh", "build_kernel.cuh", "prefill_sm100.cuh", "combine_kernel.cuh",
            "mass_sm100.cuh", "topk_kernel.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
               "-Xcompiler", "-fPIC", "-shared"]

@@ -12,6 +12,7 @@
 #include <stdint.h>
 
 #include "plan.h"
+#include "rope.cuh"
 
 namespace segpaged {
 
@@ -32,23 +33,6 @@ struct BuildParams {
 
 __device__ __forceinline__ void report(int32_t* status, int32_t bit) {
   if (status) atomicOr(status, bit);
-}
-
-__device__ __forceinline__ uint32_t rot_pair(uint32_t a2, uint32_t b2, float c0, float s0, float c1, float s1,
-                                             uint32_t* out_b) {
-  // a2 holds two bf16 of the first half (d, d+1), b2 the matching two of the second half.
-  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&a2);
-  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&b2);
-  float x1a = __low2float(a), x1b = __high2float(a);
-  float x2a = __low2float(b), x2b = __high2float(b);
-  float y1a = __fsub_rn(__fmul_rn(x1a, c0), __fmul_rn(x2a, s0));
-  float y2a = __fadd_rn(__fmul_rn(x2a, c0), __fmul_rn(x1a, s0));
-  float y1b = __fsub_rn(__fmul_rn(x1b, c1), __fmul_rn(x2b, s1));
-  float y2b = __fadd_rn(__fmul_rn(x2b, c1), __fmul_rn(x1b, s1));
-  __nv_bfloat162 o1 = __halves2bfloat162(__float2bfloat16_rn(y1a), __float2bfloat16_rn(y1b));
-  __nv_bfloat162 o2 = __halves2bfloat162(__float2bfloat16_rn(y2a), __float2bfloat16_rn(y2b));
-  *out_b = *reinterpret_cast<uint32_t*>(&o2);
-  return *reinterpret_cast<uint32_t*>(&o1);
 }
 
 template <int D, bool ROPE>

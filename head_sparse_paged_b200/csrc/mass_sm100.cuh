@@ -20,7 +20,9 @@
 //              with per-element bounds only on edge pairs, running sum in packed f32x2.
 //   warp 8     producer: claims items, TMA-loads the key tile's pages once and every query tile
 //              (same map as the prefill), and gathers the 128 rows' -LSE * log2 e into shared memory
-//              (+inf LSE for rows past the query range, so they contribute exp2(-inf) = 0).
+//              (+inf LSE for rows past the query range, so they contribute exp2(-inf) = 0). Once the key
+//              tile has landed it re-aligns its rows with the prefill's gather-time RoPE fragments, if
+//              any, and releases it to the MMA warp.
 //   warp 9     MMA issuer (whole warp, one elected lane issues): S^T into one of two TMEM buffers.
 // Every wait is bounded, as in the prefill kernel.
 #pragma once
@@ -29,6 +31,7 @@
 #include <stdint.h>
 
 #include "plan.h"
+#include "rope.cuh"
 #include "sm100_ptx.cuh"
 
 namespace segpaged {
@@ -82,11 +85,12 @@ struct MassParams {
   float* part;           // [2 warpgroups][Hkv][total_q]
   int32_t total_q, num_q_heads, num_kv_heads, num_pages, log2_group;
   float scale_log2;      // softmax_scale * log2(e)
+  RopeFragments frags;   // offs == nullptr: keys are used as stored
 };
 
 struct MassShared {
   uint64_t item_full[2], item_empty[2];
-  uint64_t k_full, k_empty;
+  uint64_t k_full, k_ready, k_empty;
   uint64_t q_full[4], q_empty[4];
   uint64_t s_full[2], s_empty[2];
   uint64_t drain;
@@ -123,6 +127,7 @@ __global__ void __launch_bounds__(320, 1)
       ptx::mbar_init(&sh.q_empty[i], 5);      // MMA commit + the 4 warps that read the tile's LSE
     }
     ptx::mbar_init(&sh.k_full, 1);
+    ptx::mbar_init(&sh.k_ready, 1);
     ptx::mbar_init(&sh.k_empty, 1);
     ptx::mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -243,6 +248,25 @@ __global__ void __launch_bounds__(320, 1)
                              &sh.q_full[s]);
           q_issued = qi + 1;
         }
+        if (t == t0) {
+          // the key tile: wait until it has landed, re-align its fragment rows, release it to the MMA warp
+          if (lane == 0) go = ptx::mbar_wait(&sh.k_full, ring & 1, abort, status, kMassStatusTimeout);
+          if (!__shfl_sync(0xffffffffu, go, 0)) break;
+          if (p.frags.offs) {
+            const int32_t flo = p.frags.offs[I[M_SEQ]], fhi = p.frags.offs[I[M_SEQ] + 1];
+            if (fhi > flo) {
+              constexpr int CH = D / 16;
+              for (int xx = lane; xx < 128 * CH; xx += 32) {
+                const int r = xx / CH, c = xx % CH;
+                const int32_t f = rope_fragment_of(p.frags.start, flo, fhi, x * 128 + r);
+                if (f >= 0) rope_rotate_smem_chunk<D>(sK, r, c, p.frags.cs + (int64_t)f * D);
+              }
+              ptx::fence_proxy_async_smem();
+            }
+          }
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&sh.k_ready);
+        }
       }
       if (!go) break;
     }
@@ -271,7 +295,7 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&sh.item_empty[slot]);
       if (nt < 0) break;
-      if (!wait(&sh.k_full, ring & 1)) break;
+      if (!wait(&sh.k_ready, ring & 1)) break;
       for (int32_t t = 0; t < nt; ++t, ++qi, ++si) {
         const int s = qi % C::NQ, b = si & 1;
         if (!wait(&sh.q_full[s], (qi / C::NQ) & 1) || !wait(&sh.s_empty[b], ((si >> 1) & 1) ^ 1)) {

@@ -25,6 +25,9 @@
 //               The commit that publishes S_t(j) also covers PV_t(j-1), so when a softmax warp sees
 //               S_t(j) its O_t is stable and can be rescaled.
 //   warps 10-11 idle.
+//   warps 12-15 only with ROPE: the gather-time RoPE re-alignment. They rotate each K tile in shared
+//               memory once it lands (keys of reused fragments, from their original to their actual
+//               positions, per sequence fragment) and only then release it to the MMA warp.
 // Every wait is bounded: on a timeout the CTA raises its abort flag, reports SEGPAGED_STATUS_TIMEOUT,
 // waits (bounded) for its TMA copies and MMAs in flight, and frees its tensor memory before returning.
 #pragma once
@@ -33,6 +36,7 @@
 #include <stdint.h>
 
 #include "plan.h"
+#include "rope.cuh"
 #include "sm100_ptx.cuh"
 
 namespace segpaged {
@@ -41,7 +45,7 @@ constexpr int32_t kStatusPageId = 1;
 constexpr int32_t kStatusTimeout = 4;
 constexpr int32_t kStatusUnit = 8;
 
-template <int D, int P>
+template <int D, int P, bool ROPE = false>
 struct PrefillCfg {
   static constexpr int BM = 128;                 // rows of one query tile (positions x heads)
   static constexpr int BN = 128;                 // keys per KV tile
@@ -52,15 +56,19 @@ struct PrefillCfg {
   static constexpr int NSLOT = (D == 128) ? 5 : 10;
   static constexpr int PPT = BN / P;             // pages per KV tile
   static constexpr int SMEM_BYTES = 2 * Q_BYTES + NSLOT * TILE_BYTES + 1024;
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = ROPE ? 512 : 384;   // ROPE: a fourth warpgroup rotates K tiles
   static constexpr uint32_t TMEM_COLS = 512;     // S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D)
   static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t IDESC_O = ptx::idesc_bf16_f32(128, D, 0, 1);
   // Register split (setmaxnreg): 256 softmax threads x 208 + 128 other threads x 80 = 63488, within the
-  // 384 x 168 = 64512 registers the block is launched with.
-  static constexpr int REGS_SOFTMAX = 208;
-  static constexpr int REGS_OTHER = 80;
-  static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= 384 * 168, "register split exceeds the launch budget");
+  // 384 x 168 = 64512 registers the block is launched with; with ROPE 256 x 192 + 128 x 64 (producer,
+  // MMA) + 128 x 64 (RoPE warpgroup) = 65536 = 512 x 128.
+  static constexpr int REGS_SOFTMAX = ROPE ? 192 : 208;
+  static constexpr int REGS_OTHER = ROPE ? 64 : 80;
+  static constexpr int REGS_ROPE = 64;
+  static constexpr int LAUNCH_REGS = ROPE ? 128 : 168;
+  static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER + (ROPE ? 128 * REGS_ROPE : 0) <= THREADS * LAUNCH_REGS,
+                "register split exceeds the launch budget");
 };
 
 struct PrefillParams {
@@ -76,7 +84,10 @@ struct PrefillParams {
   float* part_lse;       // [partial slots][256 rows] fp32: LSE of that chunk (natural log)
   int32_t total_q, num_q_heads, num_pages, log2_group;
   float scale_log2;      // softmax_scale * log2(e)
+  RopeFragments frags;   // used by the ROPE variant only
 };
+
+constexpr int kRopeSmemFragments = 256;   // fragment starts of a sequence cached in shared memory
 
 struct PrefillShared {
   uint64_t unit_full[2], unit_empty[2];
@@ -84,7 +95,9 @@ struct PrefillShared {
   uint64_t s_full[2], p_half[2], p_full[2], o_full[2], o_free[2];
   uint64_t mma_drain;
   uint64_t kv_full[10], kv_empty[10];
+  uint64_t k_rot[10];      // ROPE: K tile of tile count n rotated (ring over n % NSLOT), ready for the MMA
   __align__(16) int32_t unit[2][U_NFIELDS];
+  int32_t frag_start[kRopeSmemFragments];   // ROPE: the current unit's sequence fragment starts
   uint32_t tmem_base;
   int abort;
 };
@@ -98,11 +111,11 @@ __device__ __forceinline__ int32_t unit_logical_page(const int32_t* u, int32_t i
   return idx < u[U_NSINK] ? idx : u[U_W0] + (idx - u[U_NSINK]);
 }
 
-template <int D, int P>
-__global__ void __launch_bounds__(384, 1)
+template <int D, int P, bool ROPE>
+__global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
     segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
-  using C = PrefillCfg<D, P>;
+  using C = PrefillCfg<D, P, ROPE>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ PrefillShared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,7 +129,7 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sh.unit_full[i], 1);
-      ptx::mbar_init(&sh.unit_empty[i], 9);   // MMA lane 0 + 8 softmax warps
+      ptx::mbar_init(&sh.unit_empty[i], ROPE ? 13 : 9);   // MMA warp + 8 softmax warps (+ 4 RoPE warps)
       ptx::mbar_init(&sh.s_full[i], 1);
       ptx::mbar_init(&sh.p_half[i], 4);
       ptx::mbar_init(&sh.p_full[i], 4);
@@ -129,6 +142,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < C::NSLOT; ++i) {
       ptx::mbar_init(&sh.kv_full[i], 1);
       ptx::mbar_init(&sh.kv_empty[i], 1);
+      ptx::mbar_init(&sh.k_rot[i], 4);
     }
     sh.abort = 0;
     ptx::mbar_fence_init();
@@ -155,7 +169,8 @@ __global__ void __launch_bounds__(384, 1)
   const int npos = C::BM >> p.log2_group;    // positions per query tile
 
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
+    if (warp < 12) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
+    else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_ROPE));
     if (warp == 8) {
       // ---------------------------------------------------------------------------- producer
       // The whole warp walks the schedule; lane 0 does the barrier and TMA work, and the 32 lanes fetch
@@ -326,7 +341,11 @@ __global__ void __launch_bounds__(384, 1)
           kv_item += 2;
           if (j > 0 && !issue_pv(0, prev_vi, j == 1)) { ok = false; break; }
           const int s = ki % C::NSLOT;
-          if (!wait(&sh.kv_full[s], (ki / C::NSLOT) & 1)) { ok = false; break; }
+          // with ROPE the K tile is released by the RoPE warps; their barrier ring counts K tiles only (a
+          // slot hosts K and V items alike, so the slot's own phase count does not apply)
+          const bool kready = ROPE ? wait(&sh.k_rot[(ki >> 1) % C::NSLOT], ((ki >> 1) / C::NSLOT) & 1)
+                                   : wait(&sh.kv_full[s], (ki / C::NSLOT) & 1);
+          if (!kready) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t kb = kv_base + s * C::TILE_BYTES;
           issue_s(0, kb);
@@ -357,6 +376,90 @@ __global__ void __launch_bounds__(384, 1)
       ptx::umma_commit(leader, &sh.mma_drain);
       ptx::mbar_wait(&sh.mma_drain, 0, nullptr, status, kStatusTimeout);
       __syncwarp();
+    } else if (ROPE && warp >= 12) {
+      // ------------------------------------------------------------------- gather-time RoPE
+      // Warps 12-15 (one per SMSP) walk the schedule like the MMA warp. Per unit they cache the sequence's
+      // fragment starts in shared memory (at most kRopeSmemFragments; more are searched in global memory).
+      // Each K tile, once landed, has the rows whose token falls in a fragment rotated in place (a thread
+      // takes one 16-byte chunk pair in D/16 rows), is fenced for the tensor core and released through
+      // k_rot.
+      constexpr int CH = D / 16;                 // chunk pairs (d, d + D/2) per row
+      const int tid = (warp - 12) * 32 + lane;   // 0 .. 127
+      const int c = tid % CH;                    // this thread's chunk pair
+      uint32_t kv_item = 0;
+      auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kStatusTimeout));
+      };
+      auto rope_bar = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };   // the four RoPE warps
+      for (uint32_t ring = 0;; ++ring) {
+        const int slot = ring & 1;
+        if (!wwait(&sh.unit_full[slot], (ring >> 1) & 1)) break;
+        const int32_t* u = sh.unit[slot];
+        const int32_t ntiles = u[U_NTILES];
+        if (ntiles < 0) {
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
+          break;
+        }
+        const int32_t t0 = u[U_T0], an = u[U_AN], b0 = u[U_B0], nsink = u[U_NSINK], w0 = u[U_W0];
+        const int32_t npages = u[U_AN] + u[U_BN];
+        const int32_t flo = p.frags.offs[u[U_SEQ]], fhi = p.frags.offs[u[U_SEQ] + 1];
+        const int32_t nfr = fhi - flo;
+        const bool in_smem = nfr <= kRopeSmemFragments;
+        rope_bar();                                // the previous unit's searches are done
+        if (in_smem)
+          for (int i = tid; i < nfr; i += 128) sh.frag_start[i] = p.frags.start[flo + i];
+        rope_bar();
+        const int32_t* fst = in_smem ? sh.frag_start : p.frags.start + flo;
+        bool ok = true;
+        for (int32_t j = 0; j < ntiles; ++j) {
+          const uint32_t ki = kv_item;
+          kv_item += 2;
+          const int s = ki % C::NSLOT;
+          if (!wwait(&sh.kv_full[s], (ki / C::NSLOT) & 1)) { ok = false; break; }
+          if (nfr > 0) {
+            uint8_t* tile = sKV + s * C::TILE_BYTES;
+            auto token_of = [&](int32_t pos, int r) {
+              const int32_t idx = pos < an ? pos : b0 + (pos - an);
+              const int32_t lp = idx < nsink ? idx : w0 + (idx - nsink);
+              return lp * P + (r % P);
+            };
+            // The tile's tokens ascend with the row (pages in logical order), so if its first and last
+            // loaded rows lie in one fragment every row does: one table chunk per thread for the tile.
+            const int32_t pos0 = (t0 + j) * C::PPT;
+            const int32_t nld = min(C::PPT, npages - pos0);        // pages of this tile that were loaded
+            const int32_t f_first = rope_fragment_of(fst, 0, nfr, token_of(pos0, 0));
+            const int32_t f_last = rope_fragment_of(fst, 0, nfr, token_of(pos0 + nld - 1, nld * P - 1));
+            if (f_first == f_last) {
+              if (f_first >= 0) {
+                const float4* t4 = reinterpret_cast<const float4*>(p.frags.cs + (int64_t)(flo + f_first) * D + 16 * c);
+                const float4 t[4] = {t4[0], t4[1], t4[2], t4[3]};
+#pragma unroll 1
+                for (int k = 0; k < CH; ++k) {
+                  const int r = tid / CH + (128 / CH) * k;
+                  if (r < nld * P) rope_rotate_smem_chunk_regs<D>(tile, r, c, t);
+                }
+              }
+            } else {
+#pragma unroll 1
+              for (int k = 0; k < CH; ++k) {
+                const int r = tid / CH + (128 / CH) * k;
+                if (r >= nld * P) continue;                // page not loaded (short last tile)
+                const int32_t f = rope_fragment_of(fst, 0, nfr, token_of(pos0 + r / P, r));
+                // scalar IEEE products and sums, as the build rotates (packed f32x2 forms were measured to
+                // differ from them by one bf16 ulp in a few keys per 10^5)
+                if (f >= 0) rope_rotate_smem_chunk<D>(tile, r, c, p.frags.cs + (int64_t)(flo + f) * D);
+              }
+            }
+            ptx::fence_proxy_async_smem();            // the rotated rows are read by the tensor core
+          }
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&sh.k_rot[(ki >> 1) % C::NSLOT]);
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
+      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));

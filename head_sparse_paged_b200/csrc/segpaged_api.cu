@@ -314,20 +314,20 @@ size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpage
 
 namespace {
 
-template <int D, int P>
+template <int D, int P, bool ROPE>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
                    int grid, cudaStream_t st) {
-  using C = PrefillCfg<D, P>;
+  using C = PrefillCfg<D, P, ROPE>;
   static bool configured[kMaxDevices] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(segpaged_prefill_kernel<D, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(segpaged_prefill_kernel<D, P, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return SEGPAGED_ERR_CUDA;
     configured[dev] = true;
   }
-  segpaged_prefill_kernel<D, P><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  segpaged_prefill_kernel<D, P, ROPE><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
 }
 
@@ -341,11 +341,11 @@ int launch_combine(const CombineParams& c, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
 }
 
-extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
-                                     const void* v_pool, const int32_t* page_table, int64_t page_table_len,
-                                     const segpaged_unit* plan, const segpaged_plan_info* info, float softmax_scale,
-                                     void* o, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
-                                     void* stream) {
+namespace {
+int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool, const void* v_pool,
+                 const int32_t* page_table, int64_t page_table_len, const segpaged_unit* plan,
+                 const segpaged_plan_info* info, float softmax_scale, const RopeFragments* frags, void* o, float* lse,
+                 void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!info) return SEGPAGED_ERR_NULL;
@@ -390,10 +390,13 @@ extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, i
   p.num_pages = dims->num_pages;
   p.log2_group = log2_int(G);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.frags = frags ? *frags : RopeFragments{nullptr, nullptr, nullptr};
   const int grid = (int)std::min<int64_t>(num_units, sms);
   rc = SEGPAGED_ERR_DIMS;
-#define SEGPAGED_LAUNCH(DD, PP) \
-  if (D == DD && P == PP) rc = launch_prefill<DD, PP>(tq, tk, tv, p, grid, st);
+#define SEGPAGED_LAUNCH(DD, PP)                                                   \
+  if (D == DD && P == PP)                                                          \
+    rc = frags ? launch_prefill<DD, PP, true>(tq, tk, tv, p, grid, st)            \
+               : launch_prefill<DD, PP, false>(tq, tk, tv, p, grid, st);
   SEGPAGED_LAUNCH(128, 16)
   SEGPAGED_LAUNCH(128, 32)
   SEGPAGED_LAUNCH(128, 64)
@@ -415,6 +418,30 @@ extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, i
   c.num_q_heads = Hq;
   c.log2_group = p.log2_group;
   return D == 128 ? launch_combine<128>(c, st) : launch_combine<64>(c, st);
+}
+}  // namespace
+
+extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
+                                     const void* v_pool, const int32_t* page_table, int64_t page_table_len,
+                                     const segpaged_unit* plan, const segpaged_plan_info* info, float softmax_scale,
+                                     void* o, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                                     void* stream) {
+  return attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len, plan, info, softmax_scale, nullptr,
+                      o, lse, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int segpaged_attn_prefill_rope(const segpaged_dims* dims, const void* q, int32_t total_q,
+                                          const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                          int64_t page_table_len, const segpaged_unit* plan,
+                                          const segpaged_plan_info* info, float softmax_scale,
+                                          const int32_t* frag_offs, const int32_t* frag_start,
+                                          const float* frag_cos_sin, void* o, float* lse, void* workspace,
+                                          size_t workspace_bytes, int32_t* status, void* stream) {
+  if (!frag_offs || !frag_start || !frag_cos_sin) return SEGPAGED_ERR_NULL;
+  if (!aligned16(frag_cos_sin)) return SEGPAGED_ERR_ALIGN;
+  const RopeFragments f{frag_offs, frag_start, frag_cos_sin};
+  return attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len, plan, info, softmax_scale, &f, o,
+                      lse, workspace, workspace_bytes, status, stream);
 }
 
 // ------------------------------------------------------------------------------------------------

@@ -111,9 +111,13 @@ int launch_mass(const CUtensorMap& tq, const CUtensorMap& tk, const MassParams& 
 
 extern "C" int segpaged_token_mass(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
                                    const int32_t* page_table, int64_t page_table_len, const segpaged_mass_item* items,
-                                   int64_t num_items, const float* lse, float softmax_scale, float* mass,
-                                   void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+                                   int64_t num_items, const float* lse, float softmax_scale,
+                                   const int32_t* frag_offs, const int32_t* frag_start, const float* frag_cos_sin,
+                                   float* mass, void* workspace, size_t workspace_bytes, int32_t* status,
+                                   void* stream) {
   int rc = check_dims(dims);
+  if ((frag_offs || frag_start || frag_cos_sin) && !(frag_offs && frag_start && frag_cos_sin)) return SEGPAGED_ERR_NULL;
+  if (frag_cos_sin && !aligned16(frag_cos_sin)) return SEGPAGED_ERR_ALIGN;
   if (rc) return rc;
   if (num_items < 0 || num_items > INT32_MAX || total_q < 0 || page_table_len < 0) return SEGPAGED_ERR_DIMS;
   if (total_q == 0) return SEGPAGED_OK;
@@ -153,6 +157,7 @@ extern "C" int segpaged_token_mass(const segpaged_dims* dims, const void* q, int
     p.num_pages = dims->num_pages;
     p.log2_group = log2_int(G);
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.frags = RopeFragments{frag_offs, frag_start, frag_cos_sin};
     const int grid = (int)std::min<int64_t>(num_items, sms);
     rc = SEGPAGED_ERR_DIMS;
 #define SEGPAGED_LAUNCH(DD, PP) \

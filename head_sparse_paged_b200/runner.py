@@ -49,10 +49,12 @@ class Runner:
     class maps and queries -- for many-layer workloads whose dense K/V would not fit in memory at once.
     keep_dense: keep each layer's dense K/V on the device after set-up (tests compare against them).
     mass: also plan and hold the per-token attention mass (the sparse-FFN score) of every layer.
+    frags: gather-time RoPE fragments (frag_offs [B+1], frag_start [F], frag_cos_sin [F, D/2, 2] numpy arrays):
+    the pools keep the keys as drawn and prefill and token mass re-align them per fragment as they load them.
     """
 
     def __init__(self, w: synth.Workload, device="cuda", layers=None, keep_dense=False, page_seed_offset=0,
-                 shared_dense=False, split_ctas=None, mass=False):
+                 shared_dense=False, split_ctas=None, mass=False, frags=None):
         self.w = w
         self.device = torch.device(device)
         # long units are split across CTAs when one alone exceeds a CTA's share (short query ranges)
@@ -91,9 +93,17 @@ class Runner:
         self.mass_workspace = None
         self.with_mass = mass
         self.cu_q_dev = torch.from_numpy(w.cu_q().astype(np.int32)).to(self.device)
+        self.frags = None
+        if frags is not None:
+            fo, fs, fc = frags
+            self.frags = (torch.from_numpy(np.ascontiguousarray(fo, dtype=np.int32)).to(self.device),
+                          torch.from_numpy(np.ascontiguousarray(fs, dtype=np.int32)).to(self.device),
+                          torch.from_numpy(np.ascontiguousarray(fc, dtype=np.float32)).to(self.device))
         self.rope = None
         if w.rope_theta is not None:
             self.rope = torch.from_numpy(sp.segpaged_rope_cos_sin(w.rope_theta, w.rope_deltas, D)).to(self.device)
+        if self.frags is not None:
+            self.rope = None          # the pools keep the keys as drawn; prefill re-aligns them per fragment
         self.scale = 1.0 / math.sqrt(D)
         for li in self.layers:
             self._setup_layer(li)
@@ -173,6 +183,10 @@ class Runner:
 
     def prefill(self, li, stream=None):
         st = self.state[li]
+        if self.frags is not None:
+            sp.segpaged_attn_prefill_rope(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info,
+                                          self.scale, *self.frags, st.o, st.lse, self.workspace, self.status, stream)
+            return
         sp.segpaged_attn_prefill(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info,
                                  self.scale, st.o, st.lse, self.workspace, self.status, stream)
 
@@ -186,7 +200,7 @@ class Runner:
         """Attention mass each query row's token receives (needs this layer's prefill LSE)."""
         st = self.state[li]
         sp.segpaged_token_mass(self.dims, st.q, self.k_pool, st.table_dev, st.mass_items_dev, st.lse, self.scale, st.mass,
-                               self.mass_workspace, self.status, stream)
+                               self.mass_workspace, self.status, stream, frags=self.frags)
 
     def select_topk(self, li, k_per_seq: torch.Tensor, selected: torch.Tensor, stream=None):
         """Top-k rows per sequence by this layer's mass into `selected`."""

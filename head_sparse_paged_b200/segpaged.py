@@ -26,7 +26,7 @@ STATUS_UNIT = 8
 # Every function include/segpaged.h declares.
 EXPORTS = ("segpaged_error_string", "segpaged_pages_bytes", "segpaged_rope_cos_sin", "segpaged_build",
            "segpaged_prefill_plan", "segpaged_prefill_workspace_bytes", "segpaged_attn_prefill",
-           "segpaged_attn_prefill_noalloc", "segpaged_mass_plan", "segpaged_mass_workspace_bytes",
+           "segpaged_attn_prefill_rope", "segpaged_attn_prefill_noalloc", "segpaged_mass_plan", "segpaged_mass_workspace_bytes",
            "segpaged_token_mass", "segpaged_select_topk")
 
 
@@ -80,6 +80,9 @@ def _load():
     lib.segpaged_attn_prefill.restype = ctypes.c_int
     lib.segpaged_attn_prefill.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, ip, ctypes.c_float, vp, vp, vp,
                                           ctypes.c_size_t, vp, vp]
+    lib.segpaged_attn_prefill_rope.restype = ctypes.c_int
+    lib.segpaged_attn_prefill_rope.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, ip, ctypes.c_float, vp, vp, vp, vp, vp, vp,
+                                               ctypes.c_size_t, vp, vp]
     lib.segpaged_attn_prefill_noalloc.restype = ctypes.c_int
     lib.segpaged_attn_prefill_noalloc.argtypes = [dp, vp, i32, vp, vp, vp, i64, vp, i64, ctypes.c_float, vp, vp, vp, vp]
     lib.segpaged_mass_plan.restype = i64
@@ -87,8 +90,8 @@ def _load():
     lib.segpaged_mass_workspace_bytes.restype = ctypes.c_size_t
     lib.segpaged_mass_workspace_bytes.argtypes = [dp, i32]
     lib.segpaged_token_mass.restype = ctypes.c_int
-    lib.segpaged_token_mass.argtypes = [dp, vp, i32, vp, vp, i64, vp, i64, vp, ctypes.c_float, vp, vp, ctypes.c_size_t,
-                                        vp, vp]
+    lib.segpaged_token_mass.argtypes = [dp, vp, i32, vp, vp, i64, vp, i64, vp, ctypes.c_float, vp, vp, vp, vp, vp,
+                                        ctypes.c_size_t, vp, vp]
     lib.segpaged_select_topk.restype = ctypes.c_int
     lib.segpaged_select_topk.argtypes = [i32, vp, vp, vp, vp, vp]
     return lib
@@ -216,6 +219,25 @@ def segpaged_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, plan, info:
         raise SegPagedError(r, "segpaged_attn_prefill")
 
 
+def segpaged_attn_prefill_rope(dims: Dims, q, k_pool, v_pool, page_table, plan, info: dict, softmax_scale, frag_offs,
+                               frag_start, frag_cos_sin, o, lse, workspace, status=None, stream=None):
+    """segpaged_attn_prefill with gather-time RoPE re-alignment per sequence fragment. frag_offs int32 [B+1],
+    frag_start int32 [F], frag_cos_sin float32 [F, D/2, 2] (CUDA tensors)."""
+    bf = torch.bfloat16
+    r = _lib.segpaged_attn_prefill_rope(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]),
+                                        _dev(k_pool, bf, "k_pool"), _dev(v_pool, bf, "v_pool"),
+                                        _dev(page_table, torch.int32, "page_table"), int(page_table.numel()),
+                                        _dev(plan, torch.int32, "plan"), ctypes.byref(_info(info)), float(softmax_scale),
+                                        _dev(frag_offs, torch.int32, "frag_offs"),
+                                        _dev(frag_start, torch.int32, "frag_start"),
+                                        _dev(frag_cos_sin, torch.float32, "frag_cos_sin"), _dev(o, bf, "o"),
+                                        _dev(lse, torch.float32, "lse"), _dev(workspace, None, "workspace"),
+                                        int(workspace.numel() * workspace.element_size()),
+                                        _dev(status, torch.int32, "status"), _stream(stream))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_attn_prefill_rope")
+
+
 NOALLOC_MAX_UNITS = 16384
 
 
@@ -258,14 +280,18 @@ def segpaged_mass_workspace_bytes(dims: Dims, total_q: int) -> int:
 
 
 def segpaged_token_mass(dims: Dims, q, k_pool, page_table, items, lse, softmax_scale, mass, workspace, status=None,
-                        stream=None):
+                        stream=None, frags=None):
     """mass [total_q] float32 (CUDA), written in place: the attention mass each query row's token receives.
-    items: the mass plan on the device; lse: the prefill's LSE [Hq, total_q] for the same inputs."""
+    items: the mass plan on the device; lse: the prefill's LSE [Hq, total_q] for the same inputs; frags:
+    (frag_offs, frag_start, frag_cos_sin) of a gather-time RoPE prefill, or None."""
     bf = torch.bfloat16
+    fo, fs, fc = frags if frags is not None else (None, None, None)
     r = _lib.segpaged_token_mass(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]), _dev(k_pool, bf, "k_pool"),
                                  _dev(page_table, torch.int32, "page_table"), int(page_table.numel()),
                                  _dev(items, torch.int32, "items"), int(items.shape[0]), _dev(lse, torch.float32, "lse"),
-                                 float(softmax_scale), _dev(mass, torch.float32, "mass"),
+                                 float(softmax_scale), _dev(fo, torch.int32, "frag_offs"),
+                                 _dev(fs, torch.int32, "frag_start"), _dev(fc, torch.float32, "frag_cos_sin"),
+                                 _dev(mass, torch.float32, "mass"),
                                  _dev(workspace, None, "workspace"), int(workspace.numel() * workspace.element_size()),
                                  _dev(status, torch.int32, "status"), _stream(stream))
     if r < 0:

@@ -192,6 +192,28 @@ int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t tota
                           int32_t* status, void* stream);
 
 /*
+ * EXECUTE with the RoPE re-alignment applied at gather time instead of at build time, so a sequence can
+ * hold many reused fragments whose keys were computed at other offsets (shshi.cn, 技术原理 2
+ * "位置无关缓存复用", item "RoPE位置对齐"). The pools hold the keys as computed offline; each K tile is
+ * rotated in shared memory after it lands and before the logits are formed. Arguments as
+ * segpaged_attn_prefill, plus (all dev):
+ *   frag_offs (int32) [B+1]: sequence b owns fragments [frag_offs[b], frag_offs[b+1]);
+ *   frag_start (int32): token position where each fragment starts, ascending within a sequence;
+ *   frag_cos_sin (float, 16-byte aligned) [num_fragments][D/2][2]: the fragment's table for its shift
+ *     delta = actual - original position, as segpaged_rope_cos_sin computes it.
+ * A key token is rotated with the table of the last fragment of its sequence that starts at or before it;
+ * tokens before the first fragment keep their keys. The rotation is the build's (same rounding), so one
+ * fragment per sequence starting at 0 gives bit-identical results to segpaged_build with that table
+ * followed by segpaged_attn_prefill. V is never rotated.
+ */
+int segpaged_attn_prefill_rope(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
+                               const void* v_pool, const int32_t* page_table, int64_t page_table_len,
+                               const segpaged_unit* plan, const segpaged_plan_info* info, float softmax_scale,
+                               const int32_t* frag_offs, const int32_t* frag_start, const float* frag_cos_sin,
+                               void* o, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                               void* stream);
+
+/*
  * segpaged_attn_prefill without caller-provided device scratch. The paper has no counterpart: this
  * entry point exists for callers that cannot allocate device memory when they run prefill (for
  * example code inside a framework's own memory pool, or a runtime that forbids allocation on its
@@ -242,7 +264,7 @@ int64_t segpaged_mass_plan(const segpaged_dims* dims, const int32_t* ctx_len, co
                            const segpaged_head_class* cls, const int32_t* page_table_offs,
                            segpaged_mass_item* items, int64_t capacity);
 
-/* Device workspace segpaged_token_mass needs: one partial sum per (KV head, query row) and a counter. */
+/* Device workspace segpaged_token_mass needs: two partial sums per (KV head, query row) and a counter. */
 size_t segpaged_mass_workspace_bytes(const segpaged_dims* dims, int32_t total_q);
 
 /*
@@ -251,12 +273,15 @@ size_t segpaged_mass_workspace_bytes(const segpaged_dims* dims, int32_t total_q)
  * normalises them with `lse`, the natural-log LSE [Hq, total_q] (dev, float32) that
  * segpaged_attn_prefill wrote for the same q, pools and scale. Same q, pools, page table and scale
  * as that prefill. items (dev) [num_items] from segpaged_mass_plan; workspace (dev, 256-byte
- * aligned) of segpaged_mass_workspace_bytes. The sum over KV heads is taken in a fixed order, so
- * the result does not depend on scheduling or on the physical page ids. Asynchronous on `stream`.
+ * aligned) of segpaged_mass_workspace_bytes. frag_offs, frag_start, frag_cos_sin (dev, all NULL or
+ * all set): the fragments of a prefill run with segpaged_attn_prefill_rope, whose keys are re-aligned
+ * the same way here. The sum over KV heads is taken in a fixed order, so the result does not depend on
+ * scheduling or on the physical page ids. Asynchronous on `stream`.
  */
 int segpaged_token_mass(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,
                         const int32_t* page_table, int64_t page_table_len, const segpaged_mass_item* items,
-                        int64_t num_items, const float* lse, float softmax_scale, float* mass, void* workspace,
+                        int64_t num_items, const float* lse, float softmax_scale, const int32_t* frag_offs,
+                        const int32_t* frag_start, const float* frag_cos_sin, float* mass, void* workspace,
                         size_t workspace_bytes, int32_t* status, void* stream);
 
 /*
