@@ -51,6 +51,8 @@ def parse_args(argv=None):
                     help="skip the token-mass / top-k selection measurement (sparse-FFN score)")
     ap.add_argument("--no-rope-gather", action="store_true",
                     help="skip the gather-time RoPE measurement (prefill with per-fragment key re-alignment)")
+    ap.add_argument("--no-append", action="store_true",
+                    help="skip the fused append-and-attend measurement")
     ap.add_argument("--fragment-tokens", type=int, default=4096,
                     help="tokens per reused fragment in the gather-time RoPE measurement")
     ap.add_argument("--topk-frac", type=float, default=0.25,
@@ -464,6 +466,9 @@ def run_ours(args, rank, world, local):
     rope_gather = None
     if not args.no_rope_gather and runner.rope is None:
         rope_gather = measure_rope_gather(runner, args, device, flops_layer, prefill_total_ms / args.steps)
+    append = None
+    if not args.no_append and runner.rope is None:
+        append = measure_append(runner, args, device, flops_layer, prefill_total_ms / args.steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -497,6 +502,7 @@ def run_ours(args, rank, world, local):
         "e2e": e2e,
         "token_mass": mass,
         "rope_gather": rope_gather,
+        "append": append,
         "gpu_launches": args.steps * n_layers * 2,
         "clocks": clocks,
     }
@@ -612,6 +618,62 @@ def measure_rope_gather(runner, args, device, flops_layer, plain_prefill_ms_per_
     return {"kernel": "segpaged_prefill_kernel<ROPE>", "fragment_tokens": args.fragment_tokens,
             "fragments": len(starts), "prefill_ms_per_layer": ms / len(ev),
             "tflops": flops / (ms * 1e-3) / 1e12, "time_vs_plain_prefill": per_step / plain_prefill_ms_per_step}
+
+
+def measure_append(runner, args, device, flops_layer, plain_prefill_ms_per_step):
+    """Fused append-and-attend for every layer: the query rows' keys and values (gathered from the layer's
+    dense K/V) are written into their pool pages by the same launch that attends over them. The pool
+    already holds those rows, so the measurement leaves it unchanged. CUDA events around each launch."""
+    import numpy as np
+    import torch
+    from head_sparse_paged_b200 import segpaged as sp
+    w = runner.w
+    ck = w.cu_k()
+    rows = torch.cat([torch.arange(int(ck[b + 1]) - w.q_lens[b], int(ck[b + 1]), device=device)
+                      for b in range(w.num_seqs)])
+    plans, news = {}, {}
+    ws = runner.workspace
+    for li in runner.layers:
+        st = runner.state[li]
+        units, info = sp.segpaged_prefill_plan_append(runner.dims, runner.ctx, runner.ql, st.cls, st.offs,
+                                                      runner.split_ctas)
+        plans[li] = (torch.from_numpy(np.ascontiguousarray(units)).to(device), info)
+        need = sp.segpaged_prefill_workspace_bytes(runner.dims, info)
+        if ws.numel() * 4 < need:
+            ws = torch.zeros((need + 3) // 4, dtype=torch.int32, device=device)
+        key = 0 if runner.shared_dense else li
+        if key not in news:
+            k, v = runner.dense_of(li)
+            news[key] = (k[rows].contiguous(), v[rows].contiguous())
+    stream = torch.cuda.current_stream()
+
+    def call(li):
+        st = runner.state[li]
+        kn, vn = news[0 if runner.shared_dense else li]
+        sp.segpaged_attn_prefill_append(runner.dims, st.q, kn, vn, runner.k_pool, runner.v_pool, st.table_dev,
+                                        plans[li][0], plans[li][1], runner.scale, st.o, st.lse, ws, runner.status)
+
+    for _ in range(args.warmup):
+        for li in runner.layers:
+            call(li)
+    torch.cuda.synchronize()
+    ev = []
+    for _ in range(args.steps):
+        for li in runner.layers:
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call(li)
+            b.record(stream)
+            ev.append((li, a, b))
+    torch.cuda.synchronize()
+    runner.check_status()
+    ms = sum(a.elapsed_time(b) for _, a, b in ev)
+    flops = sum(flops_layer[li] for li, _, _ in ev)
+    return {"kernel": "segpaged_prefill_kernel<append>", "prefill_ms_per_layer": ms / len(ev),
+            "tflops": flops / (ms * 1e-3) / 1e12,
+            "appended_bytes_per_layer": 2 * int(rows.numel()) * w.num_kv_heads * w.head_dim * 2,
+            "time_vs_plain_prefill": (ms / args.steps) / plain_prefill_ms_per_step}
 
 
 def measure_e2e(runner, args, world, device, flops_step):

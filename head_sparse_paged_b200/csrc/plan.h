@@ -76,6 +76,15 @@ enum UnitField {
   U_PART = 17,    // partial slot written by a chunk of a split unit, -1 when the record writes O directly
   U_HALF = 18,    // 1 when the second query tile has no valid rows
   U_NSPLIT = 19,  // chunks of the unit (combine records)
+  // Fused append-and-attend (segpaged_attn_prefill_append). The list above then holds only the pages with
+  // a key before the query range (split at q0), forming tiles [0, n_old_tiles); tiles from n_old_tiles on
+  // cover the new pages new0 .. new0 + n_new - 1, whose rows are read from the dense new K/V instead of
+  // the pool. Keys are valid in an old tile only below `split_q0` and in a new tile only from it.
+  U_NOLDT = 20,   // tiles over the page list; the rest are new-page tiles (== U_NTILES without append)
+  U_NEW0 = 21,    // first new logical page
+  U_NNEW = 22,    // new pages (0 without append)
+  U_SPLITQ = 23,  // q0 with append, INT32_MAX without (every listed key is valid)
+  U_CUQ = 24,     // packed row of the sequence's first query (row of key position q0 in the new K/V)
   U_NFIELDS = 32
 };
 // A combine record reuses U_QROW, U_NPOS, U_KVH, U_SEQ, U_HALF; U_PART is its first partial slot and

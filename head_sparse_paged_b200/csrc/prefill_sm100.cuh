@@ -24,7 +24,8 @@
 //               TMEM, V MN-major from shared memory; keys 0-63 as soon as that half of P is written).
 //               The commit that publishes S_t(j) also covers PV_t(j-1), so when a softmax warp sees
 //               S_t(j) its O_t is stable and can be rescaled.
-//   warps 10-11 idle.
+//   warps 10-11 idle, or when appending (fused append-and-attend) writing the new keys and values of the
+//               unit's query positions into their pool pages.
 //   warps 12-15 only with ROPE: the gather-time RoPE re-alignment. They rotate each K tile in shared
 //               memory once it lands (keys of reused fragments, from their original to their actual
 //               positions, per sequence fragment) and only then release it to the MMA warp.
@@ -85,10 +86,19 @@ struct PrefillParams {
   int32_t total_q, num_q_heads, num_pages, log2_group;
   float scale_log2;      // softmax_scale * log2(e)
   RopeFragments frags;   // used by the ROPE variant only
+  // fused append-and-attend: the new keys/values [total_q, Hkv, D] are read for the new-page tiles and
+  // written into their pool pages by warps 10-11
+  int32_t append;
+  int32_t num_kv_heads;
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_pool;
+  __nv_bfloat16* v_pool;
 };
 
 constexpr int kRopeSmemFragments = 256;   // fragment starts of a sequence cached in shared memory
 
+template <bool ROPE>
 struct PrefillShared {
   uint64_t unit_full[2], unit_empty[2];
   uint64_t q_full, q_empty;
@@ -97,7 +107,7 @@ struct PrefillShared {
   uint64_t kv_full[10], kv_empty[10];
   uint64_t k_rot[10];      // ROPE: K tile of tile count n rotated (ring over n % NSLOT), ready for the MMA
   __align__(16) int32_t unit[2][U_NFIELDS];
-  int32_t frag_start[kRopeSmemFragments];   // ROPE: the current unit's sequence fragment starts
+  int32_t frag_start[ROPE ? kRopeSmemFragments : 1];   // ROPE: the current unit's sequence fragment starts
   uint32_t tmem_base;
   int abort;
 };
@@ -111,13 +121,18 @@ __device__ __forceinline__ int32_t unit_logical_page(const int32_t* u, int32_t i
   return idx < u[U_NSINK] ? idx : u[U_W0] + (idx - u[U_NSINK]);
 }
 
-template <int D, int P, bool ROPE>
-__global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
+// Kernel variants: the plain prefill, gather-time RoPE, and fused append-and-attend.
+constexpr int kModePlain = 0, kModeRope = 1, kModeAppend = 2;
+
+template <int D, int P, int MODE>
+__global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                            const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
+                            const __grid_constant__ CUtensorMap tm_vn, const PrefillParams p) {
+  constexpr bool ROPE = MODE == kModeRope, APPEND = MODE == kModeAppend;
   using C = PrefillCfg<D, P, ROPE>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ PrefillShared sh;
+  __shared__ PrefillShared<ROPE> sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                        // 2 query tiles x Q_BYTES
   uint8_t* sKV = smem + 2 * C::Q_BYTES;      // NSLOT x TILE_BYTES
@@ -129,7 +144,8 @@ __global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sh.unit_full[i], 1);
-      ptx::mbar_init(&sh.unit_empty[i], ROPE ? 13 : 9);   // MMA warp + 8 softmax warps (+ 4 RoPE warps)
+      // MMA warp + 8 softmax warps (+ 4 RoPE warps, or + 2 append warps)
+      ptx::mbar_init(&sh.unit_empty[i], ROPE ? 13 : (APPEND ? 11 : 9));
       ptx::mbar_init(&sh.s_full[i], 1);
       ptx::mbar_init(&sh.p_half[i], 4);
       ptx::mbar_init(&sh.p_full[i], 4);
@@ -151,6 +167,10 @@ __global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
     ptx::tma_prefetch_desc(&tm_q);
     ptx::tma_prefetch_desc(&tm_k);
     ptx::tma_prefetch_desc(&tm_v);
+    if (APPEND) {
+      ptx::tma_prefetch_desc(&tm_kn);
+      ptx::tma_prefetch_desc(&tm_vn);
+    }
   }
   if (warp == 9) {
     ptx::tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
@@ -216,34 +236,47 @@ __global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
         const int32_t t0 = U[U_T0];
         const int32_t ntiles = U[U_NTILES];
         const int64_t toff = U[U_TOFF];
+        const int32_t noldt = U[U_NOLDT], new0 = U[U_NEW0], nnew = U[U_NNEW];
+        const int32_t kvh = U[U_KVH], newrow0 = U[U_CUQ] - U[U_SPLITQ];   // new-K/V row of key position 0
+        if (nnew > 0 && !APPEND && lane == 0 && status) atomicOr(status, kStatusUnit);   // append plan, plain call
         int32_t batch = -1, my_pid = -1;   // page id of list position 32 * batch + lane (-1: none)
         int ok = 1;
         for (int32_t j = t0; j < t0 + ntiles && ok; ++j) {
-          const int32_t x0 = j * C::PPT;     // a tile's PPT positions never straddle a batch of 32
-          if ((x0 >> 5) != batch) {
-            batch = x0 >> 5;
-            const int32_t x = (batch << 5) + lane;
-            my_pid = -1;
-            if (x < npages) {
-              const int32_t idx = unit_table_index(U, x);
-              my_pid = 0;
-              if (idx < 0 || idx >= U[U_TOTAL] || toff + idx >= p.page_table_len) {
-                if (status) atomicOr(status, kStatusUnit);
-              } else {
-                my_pid = p.page_table[toff + idx];
-                if (my_pid < 0 || my_pid >= p.num_pages) {
-                  if (status) atomicOr(status, kStatusPageId);
-                  my_pid = 0;
+          int32_t pages[C::PPT];             // physical page ids (pool tiles) or logical pages (new-page tiles)
+          int32_t n_ok = 0;
+          const bool fresh = APPEND && j >= noldt;
+          if (!fresh) {
+            const int32_t x0 = j * C::PPT;     // a tile's PPT positions never straddle a batch of 32
+            if ((x0 >> 5) != batch) {
+              batch = x0 >> 5;
+              const int32_t x = (batch << 5) + lane;
+              my_pid = -1;
+              if (x < npages) {
+                const int32_t idx = unit_table_index(U, x);
+                my_pid = 0;
+                if (idx < 0 || idx >= U[U_TOTAL] || toff + idx >= p.page_table_len) {
+                  if (status) atomicOr(status, kStatusUnit);
+                } else {
+                  my_pid = p.page_table[toff + idx];
+                  if (my_pid < 0 || my_pid >= p.num_pages) {
+                    if (status) atomicOr(status, kStatusPageId);
+                    my_pid = 0;
+                  }
                 }
               }
             }
-          }
-          int32_t pages[C::PPT];
-          int32_t n_ok = 0;
 #pragma unroll
-          for (int c = 0; c < C::PPT; ++c) {
-            pages[c] = __shfl_sync(0xffffffffu, my_pid, (x0 + c) & 31);
-            n_ok += pages[c] >= 0 ? 1 : 0;
+            for (int c = 0; c < C::PPT; ++c) {
+              pages[c] = __shfl_sync(0xffffffffu, my_pid, (x0 + c) & 31);
+              n_ok += pages[c] >= 0 ? 1 : 0;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < C::PPT; ++c) {
+              const int32_t xn = (j - noldt) * C::PPT + c;
+              pages[c] = xn < nnew ? new0 + xn : -1;
+              n_ok += pages[c] >= 0 ? 1 : 0;
+            }
           }
           if (lane == 0) {
 #pragma unroll
@@ -260,9 +293,14 @@ __global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
               for (int c = 0; c < C::PPT; ++c) {
                 if (pages[c] < 0) continue;
 #pragma unroll
-                for (int h = 0; h < C::NH; ++h)
-                  ptx::tma_load_3d(dst + h * C::BLK + c * P * 128, which ? &tm_v : &tm_k, h * 64, 0, pages[c],
-                                   &sh.kv_full[s]);
+                for (int h = 0; h < C::NH; ++h) {
+                  if (!fresh)
+                    ptx::tma_load_3d(dst + h * C::BLK + c * P * 128, which ? &tm_v : &tm_k, h * 64, 0, pages[c],
+                                     &sh.kv_full[s]);
+                  else   // P rows of the new K/V from key position pages[c] * P (rows before q0 are masked)
+                    ptx::tma_load_3d(dst + h * C::BLK + c * P * 128, which ? &tm_vn : &tm_kn, h * 64, kvh,
+                                     newrow0 + pages[c] * P, &sh.kv_full[s]);
+                }
               }
               kv_issued = item + 1;
             }
@@ -376,6 +414,54 @@ __global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
       ptx::umma_commit(leader, &sh.mma_drain);
       ptx::mbar_wait(&sh.mma_drain, 0, nullptr, status, kStatusTimeout);
       __syncwarp();
+    } else if (APPEND && warp >= 10) {
+      // ------------------------------------------------------------------------------ append
+      // Warps 10-11 write the new keys and values of the unit's own query positions into their pool pages
+      // (the positions of a (sequence, KV head) are split among its units, so every new row is written
+      // once; of a split unit only the chunk that starts it writes). No CTA reads a new row from the pool:
+      // new-page tiles take them from the new K/V, and the pool tile of the page holding q0 masks them.
+      constexpr int VPR = D / 8;                 // 16-byte vectors per row
+      const int tid = (warp - 10) * 32 + lane;   // 0 .. 63
+      auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kStatusTimeout));
+      };
+      for (uint32_t ring = 0;; ++ring) {
+        const int slot = ring & 1;
+        if (!wwait(&sh.unit_full[slot], (ring >> 1) & 1)) break;
+        const int32_t* u = sh.unit[slot];
+        if (u[U_NTILES] < 0) {
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
+          break;
+        }
+        if (u[U_T0] == 0 && u[U_NNEW] > 0) {
+          const int32_t pos0 = u[U_POS0], nv = u[U_NPOS], qrow = u[U_QROW], kvh = u[U_KVH];
+          const int32_t nsink = u[U_NSINK], w0 = u[U_W0], total = u[U_TOTAL];
+          const bool is_global = u[U_GLOBAL] != 0;
+          const int64_t toff = u[U_TOFF];
+          for (int x = tid; x < 2 * nv * VPR; x += 64) {
+            const int which = x / (nv * VPR), rest = x % (nv * VPR);
+            const int32_t i = rest / VPR, vc = rest % VPR;
+            const int32_t pos = pos0 + i, lp = pos / P;
+            const int32_t idx = is_global ? lp : (lp < nsink ? lp : nsink + (lp - w0));
+            if (idx < 0 || idx >= total || toff + idx >= p.page_table_len || qrow + i >= p.total_q) {
+              if (status) atomicOr(status, kStatusUnit);
+              continue;
+            }
+            const int32_t pid = p.page_table[toff + idx];
+            if (pid < 0 || pid >= p.num_pages) {
+              if (status) atomicOr(status, kStatusPageId);
+              continue;
+            }
+            const int64_t src = ((int64_t)(qrow + i) * p.num_kv_heads + kvh) * D + vc * 8;
+            const int64_t dst = ((int64_t)pid * P + (pos % P)) * D + vc * 8;
+            *reinterpret_cast<uint4*>((which ? p.v_pool : p.k_pool) + dst) =
+                *reinterpret_cast<const uint4*>((which ? p.v_new : p.k_new) + src);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
+      }
     } else if (ROPE && warp >= 12) {
       // ------------------------------------------------------------------- gather-time RoPE
       // Warps 12-15 (one per SMSP) walk the schedule like the MMA warp. Per unit they cache the sequence's
@@ -499,26 +585,37 @@ __global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
       const int32_t S = u[U_SINK], W = u[U_WIN];
       const int32_t npages = u[U_AN] + u[U_BN];
       const int32_t an = u[U_AN], b0 = u[U_B0], nsink = u[U_NSINK], w0 = u[U_W0];
+      const int32_t noldt = u[U_NOLDT], new0 = u[U_NEW0], nnew = u[U_NNEW], splitq = u[U_SPLITQ];
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
 
       for (int32_t j = 0; j < ntiles; ++j) {
         // Logical page of every slot of this KV tile, worked out before S is ready; a row needs per-column
-        // bounds only if some key of the tile is invisible to it (causal edge, window edge, sink tail, or
-        // a short last tile).
+        // bounds only if some key of the tile is invisible to it (causal edge, window edge, sink tail, a
+        // short last tile, or -- appending -- the page holding q0, split between pool and new K/V).
+        const int32_t tt = t0 + j;
+        const bool fresh = APPEND && tt >= noldt;
         int32_t lp[C::PPT];
         bool need_mask = false;
 #pragma unroll
         for (int c = 0; c < C::PPT; ++c) {
-          const int32_t x = (t0 + j) * C::PPT + c;
-          if (x < npages) {
-            const int32_t idx = x < an ? x : b0 + (x - an);
-            lp[c] = idx < nsink ? idx : w0 + (idx - nsink);
+          lp[c] = -1;
+          if (!fresh) {
+            const int32_t x = tt * C::PPT + c;
+            if (x < npages) {
+              const int32_t idx = x < an ? x : b0 + (x - an);
+              lp[c] = idx < nsink ? idx : w0 + (idx - nsink);
+            }
+          } else {
+            const int32_t xn = (tt - noldt) * C::PPT + c;
+            if (xn < nnew) lp[c] = new0 + xn;
+          }
+          if (lp[c] >= 0) {
             const int32_t j0 = lp[c] * P, j1 = j0 + P - 1;
-            const bool all_vis = (j1 <= i_pos) && (is_global || j1 < S || j0 > i_pos - W);
+            const bool all_vis = (j1 <= i_pos) && (is_global || j1 < S || j0 > i_pos - W) &&
+                                 (!APPEND || (fresh ? j0 >= splitq : j1 < splitq));
             need_mask |= !all_vis;
           } else {
-            lp[c] = -1;
             need_mask = true;
           }
         }
@@ -547,7 +644,8 @@ __global__ void __launch_bounds__(ROPE ? 512 : 384, 1)
                 const int col = c * P + r;               // compile-time: columns outside this half skip
                 if (col < h * 64 || col >= h * 64 + 64) continue;
                 const int32_t jj = base + r;
-                const bool vis = lp[c] >= 0 && jj <= i_pos && (is_global || jj < S || jj > i_pos - W);
+                const bool vis = lp[c] >= 0 && jj <= i_pos && (is_global || jj < S || jj > i_pos - W) &&
+                                 (!APPEND || (fresh ? jj >= splitq : jj < splitq));
                 if (!vis) s[col] = -INFINITY;
               }
             }

@@ -123,9 +123,13 @@ int segpaged_build(const segpaged_dims* dims, const void* k_dense, const void* v
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
 }
 
-int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
-                              const segpaged_head_class* cls, const int32_t* page_table_offs, int32_t split_ctas,
-                              segpaged_unit* units, int64_t capacity, segpaged_plan_info* info) {
+}  // extern "C"
+
+namespace {
+// Planner of segpaged_prefill_plan (append = false) and segpaged_prefill_plan_append (append = true).
+int64_t plan_units(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                   const segpaged_head_class* cls, const int32_t* page_table_offs, int32_t split_ctas,
+                   segpaged_unit* units, int64_t capacity, segpaged_plan_info* info, bool append) {
   int rc = check_dims(dims);
   if (rc) return rc;
   const int B = dims->num_seqs, H = dims->num_kv_heads, P = dims->page_size;
@@ -150,7 +154,7 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
       const bool merged = sp.n_sink == sp.total;
       for (int32_t t0 = 0; t0 < Lq; t0 += npos) {
         const int32_t r0 = q0 + t0, nv = std::min(npos, Lq - t0), r1 = r0 + nv - 1;
-        int32_t a_n = 0, b0 = 0, b_n = 0;
+        int32_t a_n = 0, b0 = 0, b_n = 0, b_lp = 0;   // b_lp: logical page of the window part's first entry
         if (c.is_global) {
           b_n = r1 / P + 1;
         } else {
@@ -165,12 +169,28 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
             } else {
               b0 = lp_lo;
               b_n = lp_hi - lp_lo + 1;
+              b_lp = lp_lo;
             }
           } else {
             b0 = sp.n_sink + (lp_lo - sp.w0);
             b_n = lp_hi - lp_lo + 1;
+            b_lp = lp_lo;
           }
         }
+        // Append: keys before q0 come from the pool (the list truncated to pages holding such a key), keys
+        // from q0 on from the new K/V, as tiles of consecutive logical pages new0 .. new0 + n_new - 1.
+        int32_t new0 = 0, n_new = 0;
+        if (append) {
+          const int32_t qpages = (int32_t)ceil_div(q0, P);
+          a_n = std::min(a_n, qpages);
+          b_n = std::max(0, std::min(b_n, qpages - b_lp));
+          const int32_t lo_new = (c.is_global || c.sink > q0) ? q0 : std::max(q0, r0 - c.window + 1);
+          if (lo_new <= r1) {
+            new0 = lo_new / P;
+            n_new = r1 / P - new0 + 1;
+          }
+        }
+        const int32_t n_old_tiles = (int32_t)ceil_div(a_n + b_n, ppt);
         segpaged_unit u;
         std::memset(&u, 0, sizeof(u));
         u.v[U_QROW] = qrow + t0;
@@ -186,13 +206,18 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
         u.v[U_AN] = a_n;
         u.v[U_B0] = b0;
         u.v[U_BN] = b_n;
-        u.v[U_NTILES] = (int32_t)ceil_div(a_n + b_n, ppt);
+        u.v[U_NTILES] = n_old_tiles + (int32_t)ceil_div(n_new, ppt);
         u.v[U_TOTAL] = sp.total;
         u.v[U_SEQ] = b;
         u.v[U_T0] = 0;
         u.v[U_PART] = -1;
         u.v[U_HALF] = nv <= npos_tile ? 1 : 0;
         u.v[U_NSPLIT] = 0;
+        u.v[U_NOLDT] = n_old_tiles;
+        u.v[U_NEW0] = new0;
+        u.v[U_NNEW] = n_new;
+        u.v[U_SPLITQ] = append ? q0 : INT32_MAX;
+        u.v[U_CUQ] = qrow;
         out.push_back(u);
       }
     }
@@ -297,6 +322,22 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
   if (n) std::memcpy(units, out.data(), sizeof(segpaged_unit) * (size_t)n);
   return n;
 }
+}  // namespace
+
+extern "C" {
+
+int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                              const segpaged_head_class* cls, const int32_t* page_table_offs, int32_t split_ctas,
+                              segpaged_unit* units, int64_t capacity, segpaged_plan_info* info) {
+  return plan_units(dims, ctx_len, q_len, cls, page_table_offs, split_ctas, units, capacity, info, false);
+}
+
+int64_t segpaged_prefill_plan_append(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                                     const segpaged_head_class* cls, const int32_t* page_table_offs,
+                                     int32_t split_ctas, segpaged_unit* units, int64_t capacity,
+                                     segpaged_plan_info* info) {
+  return plan_units(dims, ctx_len, q_len, cls, page_table_offs, split_ctas, units, capacity, info, true);
+}
 
 namespace {
 constexpr size_t kCounterBytes = 256;
@@ -314,20 +355,20 @@ size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpage
 
 namespace {
 
-template <int D, int P, bool ROPE>
-int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
-                   int grid, cudaStream_t st) {
-  using C = PrefillCfg<D, P, ROPE>;
+template <int D, int P, int MODE>
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkn,
+                   const CUtensorMap& tvn, const PrefillParams& p, int grid, cudaStream_t st) {
+  using C = PrefillCfg<D, P, MODE == kModeRope>;
   static bool configured[kMaxDevices] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(segpaged_prefill_kernel<D, P, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(segpaged_prefill_kernel<D, P, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return SEGPAGED_ERR_CUDA;
     configured[dev] = true;
   }
-  segpaged_prefill_kernel<D, P, ROPE><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  segpaged_prefill_kernel<D, P, MODE><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tkn, tvn, p);
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
 }
 
@@ -344,8 +385,9 @@ int launch_combine(const CombineParams& c, cudaStream_t st) {
 namespace {
 int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool, const void* v_pool,
                  const int32_t* page_table, int64_t page_table_len, const segpaged_unit* plan,
-                 const segpaged_plan_info* info, float softmax_scale, const RopeFragments* frags, void* o, float* lse,
-                 void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+                 const segpaged_plan_info* info, float softmax_scale, const RopeFragments* frags, const void* k_new,
+                 const void* v_new, void* o, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
+                 void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!info) return SEGPAGED_ERR_NULL;
@@ -362,11 +404,22 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   if (total_q < 1 || dims->num_pages < 1) return SEGPAGED_ERR_DIMS;
   const int D = dims->head_dim, P = dims->page_size, Hq = dims->num_q_heads;
   const int G = Hq / dims->num_kv_heads;
-  CUtensorMap tq, tk, tv;
+  const bool append = k_new != nullptr;
+  if (append && (!aligned16(k_new) || !aligned16(v_new))) return SEGPAGED_ERR_ALIGN;
+  CUtensorMap tq, tk, tv, tkn, tvn;
   if (!encode_3d(&tq, q, D, Hq, (uint64_t)total_q, 64, G, 128 / G) ||
       !encode_3d(&tk, k_pool, D, P, (uint64_t)dims->num_pages, 64, P, 1) ||
       !encode_3d(&tv, v_pool, D, P, (uint64_t)dims->num_pages, 64, P, 1))
     return SEGPAGED_ERR_CUDA;
+  // new K/V [total_q, Hkv, D]: P-row boxes of one KV head, the same shared-memory layout as a pool page
+  if (append) {
+    if (!encode_3d(&tkn, k_new, D, dims->num_kv_heads, (uint64_t)total_q, 64, 1, P) ||
+        !encode_3d(&tvn, v_new, D, dims->num_kv_heads, (uint64_t)total_q, 64, 1, P))
+      return SEGPAGED_ERR_CUDA;
+  } else {
+    tkn = tk;
+    tvn = tv;
+  }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SEGPAGED_ERR_CUDA;
   const int sms = device_sm_count(dev);
@@ -391,12 +444,19 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   p.log2_group = log2_int(G);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.frags = frags ? *frags : RopeFragments{nullptr, nullptr, nullptr};
+  p.append = append ? 1 : 0;
+  p.num_kv_heads = dims->num_kv_heads;
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_pool = static_cast<__nv_bfloat16*>(const_cast<void*>(k_pool));
+  p.v_pool = static_cast<__nv_bfloat16*>(const_cast<void*>(v_pool));
   const int grid = (int)std::min<int64_t>(num_units, sms);
   rc = SEGPAGED_ERR_DIMS;
 #define SEGPAGED_LAUNCH(DD, PP)                                                   \
   if (D == DD && P == PP)                                                          \
-    rc = frags ? launch_prefill<DD, PP, true>(tq, tk, tv, p, grid, st)            \
-               : launch_prefill<DD, PP, false>(tq, tk, tv, p, grid, st);
+    rc = frags    ? launch_prefill<DD, PP, kModeRope>(tq, tk, tv, tkn, tvn, p, grid, st)   \
+         : append ? launch_prefill<DD, PP, kModeAppend>(tq, tk, tv, tkn, tvn, p, grid, st) \
+                  : launch_prefill<DD, PP, kModePlain>(tq, tk, tv, tkn, tvn, p, grid, st);
   SEGPAGED_LAUNCH(128, 16)
   SEGPAGED_LAUNCH(128, 32)
   SEGPAGED_LAUNCH(128, 64)
@@ -427,7 +487,18 @@ extern "C" int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, i
                                      void* o, float* lse, void* workspace, size_t workspace_bytes, int32_t* status,
                                      void* stream) {
   return attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len, plan, info, softmax_scale, nullptr,
-                      o, lse, workspace, workspace_bytes, status, stream);
+                      nullptr, nullptr, o, lse, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int segpaged_attn_prefill_append(const segpaged_dims* dims, const void* q, int32_t total_q,
+                                            const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                                            const int32_t* page_table, int64_t page_table_len,
+                                            const segpaged_unit* plan, const segpaged_plan_info* info,
+                                            float softmax_scale, void* o, float* lse, void* workspace,
+                                            size_t workspace_bytes, int32_t* status, void* stream) {
+  if (info && info->num_units > 0 && (!k_new || !v_new)) return SEGPAGED_ERR_NULL;
+  return attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len, plan, info, softmax_scale, nullptr,
+                      k_new, v_new, o, lse, workspace, workspace_bytes, status, stream);
 }
 
 extern "C" int segpaged_attn_prefill_rope(const segpaged_dims* dims, const void* q, int32_t total_q,
@@ -440,8 +511,8 @@ extern "C" int segpaged_attn_prefill_rope(const segpaged_dims* dims, const void*
   if (!frag_offs || !frag_start || !frag_cos_sin) return SEGPAGED_ERR_NULL;
   if (!aligned16(frag_cos_sin)) return SEGPAGED_ERR_ALIGN;
   const RopeFragments f{frag_offs, frag_start, frag_cos_sin};
-  return attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len, plan, info, softmax_scale, &f, o,
-                      lse, workspace, workspace_bytes, status, stream);
+  return attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len, plan, info, softmax_scale, &f,
+                      nullptr, nullptr, o, lse, workspace, workspace_bytes, status, stream);
 }
 
 // ------------------------------------------------------------------------------------------------

@@ -37,6 +37,8 @@ class LayerState:
     lse: torch.Tensor | None = None
     stored_bytes: int = 0
     dense_bytes: int = 0
+    k_new: torch.Tensor | None = None         # append: the query rows' keys / values [total_q, Hkv, D]
+    v_new: torch.Tensor | None = None
     mass_items: np.ndarray | None = None     # token-mass plan (sparse-FFN score)
     mass_items_dev: torch.Tensor | None = None
     mass: torch.Tensor | None = None
@@ -51,10 +53,13 @@ class Runner:
     mass: also plan and hold the per-token attention mass (the sparse-FFN score) of every layer.
     frags: gather-time RoPE fragments (frag_offs [B+1], frag_start [F], frag_cos_sin [F, D/2, 2] numpy arrays):
     the pools keep the keys as drawn and prefill and token mass re-align them per fragment as they load them.
+    append: fused append-and-attend -- the build writes only the rows before each query range (the query
+    rows' pool slots get unrelated values) and each prefill writes the query rows' keys/values into the pool
+    while attending over them.
     """
 
     def __init__(self, w: synth.Workload, device="cuda", layers=None, keep_dense=False, page_seed_offset=0,
-                 shared_dense=False, split_ctas=None, mass=False, frags=None):
+                 shared_dense=False, split_ctas=None, mass=False, frags=None, append=False):
         self.w = w
         self.device = torch.device(device)
         # long units are split across CTAs when one alone exceeds a CTA's share (short query ranges)
@@ -93,6 +98,9 @@ class Runner:
         self.mass_workspace = None
         self.with_mass = mass
         self.cu_q_dev = torch.from_numpy(w.cu_q().astype(np.int32)).to(self.device)
+        if append and (w.rope_theta is not None or frags is not None):
+            raise ValueError("append mode takes the new keys as given; it does not combine with RoPE re-alignment")
+        self.append = append
         self.frags = None
         if frags is not None:
             fo, fs, fc = frags
@@ -126,6 +134,14 @@ class Runner:
             else:
                 self._tmp_dense = (k, v)
         st.q = q
+        if self.append:
+            k, v = self.dense_of(li)
+            cq, ck = w.cu_q(), w.cu_k()
+            rows = torch.cat([torch.arange(int(ck[b + 1]) - w.q_lens[b], int(ck[b + 1]), device=self.device)
+                              for b in range(w.num_seqs)]) if w.total_q else torch.zeros(0, dtype=torch.long,
+                                                                                          device=self.device)
+            st.k_new = k[rows].contiguous()
+            st.v_new = v[rows].contiguous()
         st.o = torch.empty_like(q)
         st.lse = torch.empty(w.num_q_heads, w.total_q, dtype=torch.float32, device=self.device)
         self.build_layer(li)
@@ -161,7 +177,8 @@ class Runner:
     def plan_layer(self, li):
         """Host planning of one layer's work units (SELECTVISIBLESTATE)."""
         st = self.state[li]
-        st.units, st.info = sp.segpaged_prefill_plan(self.dims, self.ctx, self.ql, st.cls, st.offs, self.split_ctas)
+        plan = sp.segpaged_prefill_plan_append if self.append else sp.segpaged_prefill_plan
+        st.units, st.info = plan(self.dims, self.ctx, self.ql, st.cls, st.offs, self.split_ctas)
         return st.units
 
     def upload_plan(self, li, stream=None):
@@ -178,11 +195,25 @@ class Runner:
     def build_layer(self, li, stream=None):
         k, v = self.dense_of(li)
         st = self.state[li]
+        if self.append and st.k_new is not None:
+            # the pool gets unrelated (finite) values in the query rows: the fused prefill must overwrite them
+            w = self.w
+            ck = w.cu_k()
+            k, v = k.clone(), v.clone()
+            for b in range(w.num_seqs):
+                lo, hi = int(ck[b + 1]) - w.q_lens[b], int(ck[b + 1])
+                k[lo:hi] = -3.0 * k[lo:hi] + 1.0
+                v[lo:hi] = 0.5 * v[lo:hi] - 2.0
         sp.segpaged_build(self.dims, k, v, self.cu_k_dev, self.ql_dev, st.cls_dev, st.table_dev, st.offs_dev, self.rope,
                           self.k_pool, self.v_pool, self.status, stream)
 
     def prefill(self, li, stream=None):
         st = self.state[li]
+        if self.append:
+            sp.segpaged_attn_prefill_append(self.dims, st.q, st.k_new, st.v_new, self.k_pool, self.v_pool, st.table_dev,
+                                            st.units_dev, st.info, self.scale, st.o, st.lse, self.workspace,
+                                            self.status, stream)
+            return
         if self.frags is not None:
             sp.segpaged_attn_prefill_rope(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info,
                                           self.scale, *self.frags, st.o, st.lse, self.workspace, self.status, stream)

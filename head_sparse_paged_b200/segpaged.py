@@ -26,7 +26,8 @@ STATUS_UNIT = 8
 # Every function include/segpaged.h declares.
 EXPORTS = ("segpaged_error_string", "segpaged_pages_bytes", "segpaged_rope_cos_sin", "segpaged_build",
            "segpaged_prefill_plan", "segpaged_prefill_workspace_bytes", "segpaged_attn_prefill",
-           "segpaged_attn_prefill_rope", "segpaged_attn_prefill_noalloc", "segpaged_mass_plan", "segpaged_mass_workspace_bytes",
+           "segpaged_attn_prefill_rope", "segpaged_prefill_plan_append", "segpaged_attn_prefill_append",
+           "segpaged_attn_prefill_noalloc", "segpaged_mass_plan", "segpaged_mass_workspace_bytes",
            "segpaged_token_mass", "segpaged_select_topk")
 
 
@@ -75,6 +76,11 @@ def _load():
     ip = ctypes.POINTER(_PlanInfo)
     lib.segpaged_prefill_plan.restype = i64
     lib.segpaged_prefill_plan.argtypes = [dp, vp, vp, vp, vp, i32, vp, i64, ip]
+    lib.segpaged_prefill_plan_append.restype = i64
+    lib.segpaged_prefill_plan_append.argtypes = [dp, vp, vp, vp, vp, i32, vp, i64, ip]
+    lib.segpaged_attn_prefill_append.restype = ctypes.c_int
+    lib.segpaged_attn_prefill_append.argtypes = [dp, vp, i32, vp, vp, vp, vp, vp, i64, vp, ip, ctypes.c_float, vp, vp, vp,
+                                                 ctypes.c_size_t, vp, vp]
     lib.segpaged_prefill_workspace_bytes.restype = ctypes.c_size_t
     lib.segpaged_prefill_workspace_bytes.argtypes = [dp, ip]
     lib.segpaged_attn_prefill.restype = ctypes.c_int
@@ -179,25 +185,34 @@ def _info(d: dict) -> _PlanInfo:
     return _PlanInfo(int(d["num_units"]), int(d["num_groups"]), int(d["num_partials"]))
 
 
-def segpaged_prefill_plan(dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas: int = 0):
-    """(records int32 [n, 32], info dict). Records [0, num_units) are work units (longest first by cost
-    bucket), the rest combine records of split units. split_ctas > 0 lets long units be split across that
-    many concurrent CTAs (the SM count); 0 never splits. Host only."""
+def _plan(fn, name, dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas):
     B, H = dims.num_seqs, dims.num_kv_heads
     L, Lq = _host_i32(ctx_len, B), _host_i32(q_len, B)
     c, offs = _host_i32(cls, B * H * 3), _host_i32(page_table_offs, B * H + 1)
     d = dims.c()
     info = _PlanInfo()
-    n = _lib.segpaged_prefill_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), int(split_ctas), None, 0,
-                                   ctypes.byref(info))
+    n = fn(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), int(split_ctas), None, 0, ctypes.byref(info))
     if n < 0:
-        raise SegPagedError(int(n), "segpaged_prefill_plan")
+        raise SegPagedError(int(n), name)
     units = np.zeros((max(n, 1), UNIT_FIELDS), np.int32)
-    n2 = _lib.segpaged_prefill_plan(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), int(split_ctas), _hp(units), n,
-                                    ctypes.byref(info))
+    n2 = fn(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), int(split_ctas), _hp(units), n, ctypes.byref(info))
     if n2 < 0:
-        raise SegPagedError(int(n2), "segpaged_prefill_plan")
+        raise SegPagedError(int(n2), name)
     return units[:n], {"num_units": info.num_units, "num_groups": info.num_groups, "num_partials": info.num_partials}
+
+
+def segpaged_prefill_plan(dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas: int = 0):
+    """(records int32 [n, 32], info dict). Records [0, num_units) are work units (longest first by cost
+    bucket), the rest combine records of split units. split_ctas > 0 lets long units be split across that
+    many concurrent CTAs (the SM count); 0 never splits. Host only."""
+    return _plan(_lib.segpaged_prefill_plan, "segpaged_prefill_plan", dims, ctx_len, q_len, cls, page_table_offs,
+                 split_ctas)
+
+
+def segpaged_prefill_plan_append(dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas: int = 0):
+    """Plan of the fused append-and-attend call, same form as segpaged_prefill_plan. Host only."""
+    return _plan(_lib.segpaged_prefill_plan_append, "segpaged_prefill_plan_append", dims, ctx_len, q_len, cls,
+                 page_table_offs, split_ctas)
 
 
 def segpaged_prefill_workspace_bytes(dims: Dims, info: dict) -> int:
@@ -217,6 +232,23 @@ def segpaged_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, plan, info:
                                    _dev(status, torch.int32, "status"), _stream(stream))
     if r < 0:
         raise SegPagedError(r, "segpaged_attn_prefill")
+
+
+def segpaged_attn_prefill_append(dims: Dims, q, k_new, v_new, k_pool, v_pool, page_table, plan, info: dict,
+                                 softmax_scale, o, lse, workspace, status=None, stream=None):
+    """Fused append-and-attend: writes the query rows' new keys/values (k_new, v_new [total_q, Hkv, D] bf16)
+    into their pool pages and computes O / LSE over the pool before the query range and the new rows from it."""
+    bf = torch.bfloat16
+    r = _lib.segpaged_attn_prefill_append(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]),
+                                          _dev(k_new, bf, "k_new"), _dev(v_new, bf, "v_new"), _dev(k_pool, bf, "k_pool"),
+                                          _dev(v_pool, bf, "v_pool"), _dev(page_table, torch.int32, "page_table"),
+                                          int(page_table.numel()), _dev(plan, torch.int32, "plan"),
+                                          ctypes.byref(_info(info)), float(softmax_scale), _dev(o, bf, "o"),
+                                          _dev(lse, torch.float32, "lse"), _dev(workspace, None, "workspace"),
+                                          int(workspace.numel() * workspace.element_size()),
+                                          _dev(status, torch.int32, "status"), _stream(stream))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_attn_prefill_append")
 
 
 def segpaged_attn_prefill_rope(dims: Dims, q, k_pool, v_pool, page_table, plan, info: dict, softmax_scale, frag_offs,

@@ -163,6 +163,14 @@ int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len,
                               const segpaged_head_class* cls, const int32_t* page_table_offs, int32_t split_ctas,
                               segpaged_unit* units, int64_t capacity, segpaged_plan_info* info);
 
+/* Plans the fused append-and-attend call (segpaged_attn_prefill_append); same inputs and outputs as
+ * segpaged_prefill_plan. Each unit reads the keys before its sequence's query range from the pool and the
+ * keys from the query range on from the new K/V. Give the plan to segpaged_attn_prefill_append only. */
+int64_t segpaged_prefill_plan_append(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
+                                     const segpaged_head_class* cls, const int32_t* page_table_offs,
+                                     int32_t split_ctas, segpaged_unit* units, int64_t capacity,
+                                     segpaged_plan_info* info);
+
 /* Device scratch bytes segpaged_attn_prefill needs for a plan: the work counter and, for split plans,
  * the partial results (256 x D + 256 floats per partial slot). */
 size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpaged_plan_info* info);
@@ -190,6 +198,26 @@ int segpaged_attn_prefill(const segpaged_dims* dims, const void* q, int32_t tota
                           int64_t page_table_len, const segpaged_unit* plan, const segpaged_plan_info* info,
                           float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
                           int32_t* status, void* stream);
+
+/*
+ * EXECUTE fused with the append of the new tokens' keys and values into the pool (the online KV cache the
+ * recompute writes: aiboss88.com, 使い方, fourth item "EXECUTE" writes global-head recompute into the online
+ * KV cache), in one launch. Arguments as segpaged_attn_prefill, plus
+ *   k_new, v_new (dev) [total_q, Hkv, D] bf16, 16-byte aligned: the keys and values of the query rows
+ *     (position L - Lq + r of sequence b for row cu_q[b] + r), as the model computed them;
+ *   plan from segpaged_prefill_plan_append.
+ * Effects: every pool row of a query position of every (sequence, KV head) is overwritten with its new key
+ * and value (each exactly once), and O / LSE are the attention over the pool's rows before the query
+ * range and the new rows from it on -- the same result as segpaged_build of the full K/V followed by
+ * segpaged_attn_prefill, up to floating-point order. Pool rows of the query range are never read, so they
+ * may hold anything finite beforehand; the pages they live in must be in the page table (the storage rule
+ * keeps every page with a query position).
+ */
+int segpaged_attn_prefill_append(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_new,
+                                 const void* v_new, void* k_pool, void* v_pool, const int32_t* page_table,
+                                 int64_t page_table_len, const segpaged_unit* plan, const segpaged_plan_info* info,
+                                 float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                                 int32_t* status, void* stream);
 
 /*
  * EXECUTE with the RoPE re-alignment applied at gather time instead of at build time, so a sequence can

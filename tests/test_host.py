@@ -294,3 +294,64 @@ def test_mass_plan_covers_every_query_key_and_every_viewer(case):
         for kh in range(Hkv):
             want = set(range((L - Lq) // 128, (L - 1) // 128 + 1)) if Lq > 0 else set()
             assert {x for (bb, k, x) in got if bb == b and k == kh} == want
+
+
+# Append-mode fields (head_sparse_paged_b200/csrc/plan.h).
+U_NOLDT, U_NEW0, U_NNEW, U_SPLITQ, U_CUQ = 20, 21, 22, 23, 24
+
+
+@pytest.mark.parametrize("case", range(len(EDGE)))
+@pytest.mark.parametrize("split", [0, 1000])
+def test_append_plan_reads_old_keys_from_pool_and_new_keys_fresh(case, split):
+    """Fused append-and-attend plan: a unit's page list holds only pages with a key before q0; its new pages
+    (read from the new K/V) are consecutive logical pages from the first visible key at or after q0 to its
+    last row; together they hold every visible key of every row (the oracle's sets); rows are covered once."""
+    w_seqs, Hq, Hkv, D, P, classes = EDGE[case]
+    B = len(w_seqs)
+    dims = sp.Dims(B, Hq, Hkv, D, P)
+    ctx = [s[0] for s in w_seqs]
+    ql = [s[1] for s in w_seqs]
+    cls = np.asarray(classes, np.int32)
+    _, _, per = sp.segpaged_pages_bytes(dims, ctx, ql, cls)
+    offs = np.concatenate([[0], np.cumsum(per)]).astype(np.int32)
+    recs, info = sp.segpaged_prefill_plan_append(dims, ctx, ql, cls, offs, split)
+    units = recs[: info["num_units"]]
+    cu_q = np.concatenate([[0], np.cumsum(ql)])
+    ppt = 128 // P
+    seen = np.zeros((int(cu_q[-1]), Hkv), np.int32)
+    for u in units:
+        b, kh = int(u[U_SEQ]), int(u[U_KVH])
+        L, Lq = ctx[b], ql[b]
+        q0 = L - Lq
+        g, S, W = (int(x) for x in cls[b, kh])
+        assert u[U_SPLITQ] == q0 and u[U_CUQ] == cu_q[b]
+        npages = int(u[U_AN] + u[U_BN])
+        assert u[U_NOLDT] == -(-npages // ppt)
+        assert u[U_NTILES] == u[U_NOLDT] + -(-int(u[U_NNEW]) // ppt) or u[U_PART] >= 0
+        stored = orc.stored_logical_pages(L, Lq, bool(g), S, W, P)
+        idxs = [x if x < u[U_AN] else int(u[U_B0]) + x - int(u[U_AN]) for x in range(npages)]
+        lps = [x if x < u[U_NSINK] else int(u[U_W0]) + x - int(u[U_NSINK]) for x in idxs]
+        assert lps == [stored[x] for x in idxs]
+        assert all(lp * P < q0 for lp in lps)
+        new = list(range(int(u[U_NEW0]), int(u[U_NEW0]) + int(u[U_NNEW])))
+        covered_old = set()
+        for lp in lps:
+            covered_old.update(range(lp * P, lp * P + P))
+        covered_new = set()
+        for lp in new:
+            covered_new.update(range(lp * P, lp * P + P))
+        if u[U_PART] >= 0 and u[U_T0] != 0:
+            continue
+        for r in range(int(u[U_NPOS])):
+            i = int(u[U_POS0]) + r
+            vis = set(orc.visible_keys(bool(g), S, W, i).tolist())
+            assert {j for j in vis if j < q0} <= covered_old
+            assert {j for j in vis if j >= q0} <= covered_new
+            seen[int(u[U_QROW]) + r, kh] += 1
+        if new:
+            last = int(u[U_POS0]) + int(u[U_NPOS]) - 1
+            assert new[-1] == last // P
+            first_vis = min(j for r in range(int(u[U_NPOS])) for j in orc.visible_keys(bool(g), S, W, int(u[U_POS0]) + r)
+                            if j >= q0)
+            assert new[0] == first_vis // P
+    assert np.all(seen == 1)
