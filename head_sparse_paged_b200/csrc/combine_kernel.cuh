@@ -80,6 +80,9 @@ __global__ void __launch_bounds__(256) segpaged_combine_kernel(const CombinePara
   constexpr int NW = 8;      // warps per block
   __shared__ float s_m[NW], s_sum[NW];
   __shared__ float s_acc[NW][D];
+  // Launched as a programmatic dependent of the prefill: wait until that grid has completed and its
+  // partial results are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = 1 << p.log2_group;
   const int npos_tile = 128 >> p.log2_group;

@@ -176,10 +176,16 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     ptx::tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  // KV slots start zeroed: a partial tile leaves earlier (finite) data in the rows it does not
-  // load, and those columns are masked.
-  for (int x = threadIdx.x; x < C::NSLOT * C::TILE_BYTES / 16; x += blockDim.x)
-    reinterpret_cast<uint4*>(sKV)[x] = make_uint4(0, 0, 0, 0);
+  // KV slots start zeroed: a partial tile (pages smaller than a tile) leaves earlier (finite) data in the
+  // rows it does not load, and those columns are masked. With one page per tile every used slot is loaded
+  // whole, and the start-up saves the stores.
+  if constexpr (C::PPT > 1) {
+    for (int x = threadIdx.x; x < C::NSLOT * C::TILE_BYTES / 16; x += blockDim.x)
+      reinterpret_cast<uint4*>(sKV)[x] = make_uint4(0, 0, 0, 0);
+  }
+  // The combine launch that may follow this one (split plans) can be scheduled as SMs free up; it waits
+  // for this grid's completion before reading anything (programmatic dependent launch).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();

@@ -377,8 +377,19 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 template <int D>
 int launch_combine(const CombineParams& c, cudaStream_t st) {
   if (c.num_groups <= 0) return SEGPAGED_OK;
-  const dim3 grid((unsigned)std::min<int64_t>(c.num_groups, 65535), 256);   // records x tile rows
-  segpaged_combine_kernel<D><<<grid, 256, 0, st>>>(c);
+  // records x tile rows, as a programmatic dependent launch: its blocks are scheduled while the prefill's
+  // last CTAs finish and wait in the kernel for that grid's completion
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::min<int64_t>(c.num_groups, 65535), 256);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, segpaged_combine_kernel<D>, c) != cudaSuccess) return SEGPAGED_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
 }
 
