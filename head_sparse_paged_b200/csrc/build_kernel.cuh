@@ -104,3 +104,76 @@ __global__ void __launch_bounds__(256) build_scatter_kernel(BuildParams p) {
 }
 
 }  // namespace segpaged
+
+namespace segpaged {
+
+// Re-aligns the keys of one layer's stored pages per sequence fragment into a second K pool (the same
+// physical ids): every row whose token falls in a fragment is rotated with that fragment's table, the
+// others are copied. The prefill then reads the second pool as its K pool, so the rotation costs one
+// pass over the layer's K pages (read + write) instead of one rotation per K tile load.
+struct RealignParams {
+  const __nv_bfloat16* k_in;   // [num_pages][P][D]
+  __nv_bfloat16* k_out;        // [num_pages][P][D]
+  const int32_t* cu_k;         // [B+1]
+  const int32_t* q_len;        // [B]
+  const int32_t* cls;          // [B*Hkv][3]
+  const int32_t* table;
+  const int32_t* offs;         // [B*Hkv+1]
+  RopeFragments frags;
+  int32_t* status;
+  int32_t B, Hkv, P, num_pages;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) rope_realign_kernel(RealignParams p) {
+  constexpr int HPR = D / 16;  // vector pairs per row: (first-half chunk, second-half chunk)
+  const int nheads = p.B * p.Hkv;
+  const int64_t E = p.offs[nheads];
+  for (int64_t e = blockIdx.x; e < E; e += gridDim.x) {
+    int lo = 0, hi = nheads;  // largest head with offs[head] <= e
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.offs[mid] <= e) lo = mid; else hi = mid;
+    }
+    const int bk = lo, b = bk / p.Hkv;
+    const int32_t t = (int32_t)(e - p.offs[bk]);
+    const int32_t L = p.cu_k[b + 1] - p.cu_k[b];
+    const Split sp = storage_split(L, p.q_len[b], p.cls[3 * bk], p.cls[3 * bk + 1], p.cls[3 * bk + 2], p.P);
+    if (t >= sp.total) {
+      if (threadIdx.x == 0) report(p.status, 2);
+      continue;
+    }
+    const int32_t lp = t < sp.n_sink ? t : sp.w0 + (t - sp.n_sink);
+    const int32_t pid = p.table[e];
+    if (pid < 0 || pid >= p.num_pages) {
+      if (threadIdx.x == 0) report(p.status, 1);
+      continue;
+    }
+    const int32_t flo = p.frags.offs[b], fhi = p.frags.offs[b + 1];
+    // the page's tokens are consecutive: if its first and last lie in one fragment, so do all of them
+    const int32_t last_tok = min(lp * p.P + p.P, L) - 1;
+    const int32_t f_first = rope_fragment_of(p.frags.start, flo, fhi, lp * p.P);
+    const bool one = last_tok < lp * p.P || f_first == rope_fragment_of(p.frags.start, flo, fhi, last_tok);
+    for (int x = threadIdx.x; x < p.P * HPR; x += blockDim.x) {
+      const int row = x / HPR, pc = x % HPR;
+      const int32_t tok = lp * p.P + row;
+      const int64_t at = ((int64_t)pid * p.P + row) * D + pc * 8;
+      uint4 o1 = *reinterpret_cast<const uint4*>(p.k_in + at);
+      uint4 o2 = *reinterpret_cast<const uint4*>(p.k_in + at + D / 2);
+      const int32_t f = tok >= L ? -1 : one ? f_first : rope_fragment_of(p.frags.start, flo, fhi, tok);
+      if (f >= 0) {
+        const float4* t4 = reinterpret_cast<const float4*>(p.frags.cs + (int64_t)f * D + 2 * (pc * 8));
+        const float4 q0 = t4[0], q1 = t4[1], q2 = t4[2], q3 = t4[3];
+        const uint4 a = o1, c = o2;
+        o1.x = rot_pair(a.x, c.x, q0.x, q0.y, q0.z, q0.w, &o2.x);
+        o1.y = rot_pair(a.y, c.y, q1.x, q1.y, q1.z, q1.w, &o2.y);
+        o1.z = rot_pair(a.z, c.z, q2.x, q2.y, q2.z, q2.w, &o2.z);
+        o1.w = rot_pair(a.w, c.w, q3.x, q3.y, q3.z, q3.w, &o2.w);
+      }
+      *reinterpret_cast<uint4*>(p.k_out + at) = o1;
+      *reinterpret_cast<uint4*>(p.k_out + at + D / 2) = o2;
+    }
+  }
+}
+
+}  // namespace segpaged

@@ -326,6 +326,41 @@ int64_t plan_units(const segpaged_dims* dims, const int32_t* ctx_len, const int3
 
 extern "C" {
 
+int segpaged_rope_realign(const segpaged_dims* dims, const int32_t* cu_seqlens_k, const int32_t* q_len,
+                          const segpaged_head_class* cls, const int32_t* page_table, const int32_t* page_table_offs,
+                          const int32_t* frag_offs, const int32_t* frag_start, const float* frag_cos_sin,
+                          const void* k_pool, void* k_pool_out, int32_t* status, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->num_seqs == 0) return SEGPAGED_OK;
+  if (!cu_seqlens_k || !q_len || !cls || !page_table || !page_table_offs || !frag_offs || !frag_start ||
+      !frag_cos_sin || !k_pool || !k_pool_out)
+    return SEGPAGED_ERR_NULL;
+  if (k_pool == k_pool_out) return SEGPAGED_ERR_DIMS;
+  if (!aligned16(k_pool) || !aligned16(k_pool_out) || !aligned16(frag_cos_sin)) return SEGPAGED_ERR_ALIGN;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SEGPAGED_ERR_CUDA;
+  RealignParams p;
+  p.k_in = static_cast<const __nv_bfloat16*>(k_pool);
+  p.k_out = static_cast<__nv_bfloat16*>(k_pool_out);
+  p.cu_k = cu_seqlens_k;
+  p.q_len = q_len;
+  p.cls = reinterpret_cast<const int32_t*>(cls);
+  p.table = page_table;
+  p.offs = page_table_offs;
+  p.frags = RopeFragments{frag_offs, frag_start, frag_cos_sin};
+  p.status = status;
+  p.B = dims->num_seqs;
+  p.Hkv = dims->num_kv_heads;
+  p.P = dims->page_size;
+  p.num_pages = dims->num_pages;
+  const int grid = std::max(1, device_sm_count(dev)) * 8;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dims->head_dim == 128) rope_realign_kernel<128><<<grid, 256, 0, st>>>(p);
+  else rope_realign_kernel<64><<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
+}
+
 int64_t segpaged_prefill_plan(const segpaged_dims* dims, const int32_t* ctx_len, const int32_t* q_len,
                               const segpaged_head_class* cls, const int32_t* page_table_offs, int32_t split_ctas,
                               segpaged_unit* units, int64_t capacity, segpaged_plan_info* info) {

@@ -26,7 +26,7 @@ STATUS_UNIT = 8
 # Every function include/segpaged.h declares.
 EXPORTS = ("segpaged_error_string", "segpaged_pages_bytes", "segpaged_rope_cos_sin", "segpaged_build",
            "segpaged_prefill_plan", "segpaged_prefill_workspace_bytes", "segpaged_attn_prefill",
-           "segpaged_attn_prefill_rope", "segpaged_prefill_plan_append", "segpaged_attn_prefill_append",
+           "segpaged_attn_prefill_rope", "segpaged_rope_realign", "segpaged_prefill_plan_append", "segpaged_attn_prefill_append",
            "segpaged_attn_prefill_noalloc", "segpaged_mass_plan", "segpaged_mass_workspace_bytes",
            "segpaged_token_mass", "segpaged_select_topk")
 
@@ -76,6 +76,8 @@ def _load():
     ip = ctypes.POINTER(_PlanInfo)
     lib.segpaged_prefill_plan.restype = i64
     lib.segpaged_prefill_plan.argtypes = [dp, vp, vp, vp, vp, i32, vp, i64, ip]
+    lib.segpaged_rope_realign.restype = ctypes.c_int
+    lib.segpaged_rope_realign.argtypes = [dp] + [vp] * 12
     lib.segpaged_prefill_plan_append.restype = i64
     lib.segpaged_prefill_plan_append.argtypes = [dp, vp, vp, vp, vp, i32, vp, i64, ip]
     lib.segpaged_attn_prefill_append.restype = ctypes.c_int
@@ -249,6 +251,22 @@ def segpaged_attn_prefill_append(dims: Dims, q, k_new, v_new, k_pool, v_pool, pa
                                           _dev(status, torch.int32, "status"), _stream(stream))
     if r < 0:
         raise SegPagedError(r, "segpaged_attn_prefill_append")
+
+
+def segpaged_rope_realign(dims: Dims, cu_seqlens_k, q_len, cls, page_table, page_table_offs, frag_offs, frag_start,
+                          frag_cos_sin, k_pool, k_pool_out, status=None, stream=None):
+    """Copy one layer's stored K pages into k_pool_out (same ids) with per-fragment RoPE re-alignment."""
+    bf = torch.bfloat16
+    r = _lib.segpaged_rope_realign(ctypes.byref(dims.c()), _dev(cu_seqlens_k, torch.int32, "cu_seqlens_k"),
+                                   _dev(q_len, torch.int32, "q_len"), _dev(cls, torch.int32, "cls"),
+                                   _dev(page_table, torch.int32, "page_table"),
+                                   _dev(page_table_offs, torch.int32, "page_table_offs"),
+                                   _dev(frag_offs, torch.int32, "frag_offs"), _dev(frag_start, torch.int32, "frag_start"),
+                                   _dev(frag_cos_sin, torch.float32, "frag_cos_sin"), _dev(k_pool, bf, "k_pool"),
+                                   _dev(k_pool_out, bf, "k_pool_out"), _dev(status, torch.int32, "status"),
+                                   _stream(stream))
+    if r < 0:
+        raise SegPagedError(r, "segpaged_rope_realign")
 
 
 def segpaged_attn_prefill_rope(dims: Dims, q, k_pool, v_pool, page_table, plan, info: dict, softmax_scale, frag_offs,

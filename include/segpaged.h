@@ -220,6 +220,23 @@ int segpaged_attn_prefill_append(const segpaged_dims* dims, const void* q, int32
                                  int32_t* status, void* stream);
 
 /*
+ * The same per-fragment RoPE re-alignment as segpaged_attn_prefill_rope, done once per request instead of
+ * at every K tile load: every stored page of every (sequence, KV head) of one layer is copied from k_pool to
+ * k_pool_out at the same physical id, with the rows whose token falls in a fragment rotated (same rule,
+ * same rounding). segpaged_attn_prefill run with k_pool_out as its K pool then gives bit-identical results
+ * to segpaged_attn_prefill_rope on k_pool. One pass over the layer's K pages (read and write, HBM-bound)
+ * instead of one rotation per unit that loads a tile; it needs a second K pool (k_pool_out, dev, as large
+ * as k_pool; ids outside the layer's tables are left untouched).
+ *   cu_seqlens_k, q_len, cls, page_table, page_table_offs (dev): as for segpaged_build.
+ *   frag_offs, frag_start, frag_cos_sin (dev): as for segpaged_attn_prefill_rope.
+ * Returns SEGPAGED_ERR_DIMS if k_pool_out == k_pool.
+ */
+int segpaged_rope_realign(const segpaged_dims* dims, const int32_t* cu_seqlens_k, const int32_t* q_len,
+                          const segpaged_head_class* cls, const int32_t* page_table, const int32_t* page_table_offs,
+                          const int32_t* frag_offs, const int32_t* frag_start, const float* frag_cos_sin,
+                          const void* k_pool, void* k_pool_out, int32_t* status, void* stream);
+
+/*
  * EXECUTE with the RoPE re-alignment applied at gather time instead of at build time, so a sequence can
  * hold many reused fragments whose keys were computed at other offsets (shshi.cn, 技术原理 2
  * "位置无关缓存复用", item "RoPE位置对齐"). The pools hold the keys as computed offline; each K tile is

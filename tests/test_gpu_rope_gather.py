@@ -116,3 +116,31 @@ def test_fragment_prefill_is_bit_identical_under_page_permutation():
     b = _run(w, frags=fr, page_seed_offset=5)
     assert torch.equal(a.state[0].o, b.state[0].o) and torch.equal(a.state[0].lse, b.state[0].lse)
     assert torch.equal(a.state[0].mass, b.state[0].mass)
+
+
+@pytest.mark.parametrize("name", ["varlen-p16-g4", "mha-d64-p128", "g16-p64"])
+def test_realign_pass_then_plain_prefill_equals_gather_time_rope_bitwise(name):
+    """segpaged_rope_realign into a second K pool + the plain prefill on it == the gather-time RoPE prefill."""
+    from head_sparse_paged_b200 import segpaged as sp
+    w = SMALL[name]()
+    fr = _fragments(w, np.random.default_rng(64), per_seq=5)
+    g = _run(w, frags=fr)
+    r = Runner(w, keep_dense=True, split_ctas=g.split_ctas)
+    st = r.state[0]
+    k_out = torch.zeros_like(r.k_pool)
+    fo, fs, fc = (torch.from_numpy(np.ascontiguousarray(x)).cuda() for x in fr)
+    sp.segpaged_rope_realign(r.dims, r.cu_k_dev, r.ql_dev, st.cls_dev, st.table_dev, st.offs_dev, fo, fs, fc,
+                             r.k_pool, k_out, r.status)
+    sp.segpaged_attn_prefill(r.dims, st.q, k_out, r.v_pool, st.table_dev, st.units_dev, st.info, r.scale, st.o, st.lse,
+                             r.workspace, r.status)
+    torch.cuda.synchronize()
+    r.check_status()
+    assert torch.equal(st.o, g.state[0].o) and torch.equal(st.lse, g.state[0].lse)
+    # the re-aligned pool itself: stored pages against the oracle's re-aligned keys
+    k, v = r.dense[0]
+    kn = orc.rope_fragment_keys(k.float().cpu().numpy(), w.cu_k(), *fr)
+    c = w.classes[0]
+    kp, _ = orc.build_pool(kn, v.float().cpu().numpy(), w.cu_k(), w.cu_q(), c[..., 0], c[..., 1], c[..., 2],
+                           w.page_size, st.table, st.offs, r.num_pages)
+    used = ~np.isnan(kp[:, 0, 0])
+    np.testing.assert_array_equal(k_out.float().cpu().numpy()[used], kp[used])
