@@ -13,17 +13,17 @@
 // warpgroup owns one key's TMEM lane and sums its row: no cross-thread reduction. The sum of an item
 // goes to a per-(warpgroup, KV head, query row) partial; mass_reduce_kernel adds them in a fixed order.
 //
-// Per CTA, 10 warps:
-//   warps 0-3, 4-7  two mass warpgroups, taking the item's query tiles alternately (tile parity picks
-//              the warpgroup and its TMEM buffer), so one exponentiates while the other waits on its
-//              logits: tcgen05.ld of the key's 128 logits, exp2(s * scale * log2 e - LSE_i * log2 e)
-//              with per-element bounds only on edge pairs, running sum in packed f32x2.
-//   warp 8     producer: claims items, TMA-loads the key tile's pages once and every query tile
+// Per CTA, 14 warps:
+//   warps 0-11 three mass warpgroups, taking the item's query tiles in turn (tile number mod 3 picks the
+//              warpgroup and its TMEM buffer), so two exponentiate while the third waits on its logits:
+//              tcgen05.ld of the key's 128 logits, exp2(s * scale * log2 e - LSE_i * log2 e) with
+//              per-element bounds only on edge pairs, running sum in packed f32x2.
+//   warp 12    producer: claims items, TMA-loads the key tile's pages once and every query tile
 //              (same map as the prefill), and gathers the 128 rows' -LSE * log2 e into shared memory
 //              (+inf LSE for rows past the query range, so they contribute exp2(-inf) = 0). Once the key
 //              tile has landed it re-aligns its rows with the prefill's gather-time RoPE fragments, if
 //              any, and releases it to the MMA warp.
-//   warp 9     MMA issuer (whole warp, one elected lane issues): S^T into one of two TMEM buffers.
+//   warp 13    MMA issuer (whole warp, one elected lane issues): S^T into one of three TMEM buffers.
 // Every wait is bounded, as in the prefill kernel.
 #pragma once
 #include <cuda.h>
@@ -57,6 +57,8 @@ enum MassField : int {
   M_NFIELDS
 };
 
+constexpr int kMassWarpgroups = 3;          // warpgroups exponentiating, one TMEM buffer each
+constexpr int kMassThreads = 32 * (4 * kMassWarpgroups + 2);
 constexpr int32_t kMassStatusPageId = 1;
 constexpr int32_t kMassStatusTimeout = 4;
 constexpr int32_t kMassStatusUnit = 8;
@@ -66,11 +68,13 @@ struct MassCfg {
   static constexpr int NH = D / 64;                   // 128-byte swizzle column blocks across D
   static constexpr int BLK = 128 * 128;               // bytes of one 64-column block of a 128-row tile
   static constexpr int TILE_BYTES = 128 * D * 2;      // key tile or query tile
-  static constexpr int NQ = 4;                        // query-tile ring
+  static constexpr int NWG = kMassWarpgroups;
+  static constexpr int NQ = 5;                        // query-tile ring
   static constexpr int PPT = 128 / P;                 // pages per key tile
   static constexpr int SMEM_BYTES = TILE_BYTES * (1 + NQ) + NQ * 128 * 4 + 1024;
-  static constexpr int THREADS = 320;
-  static constexpr uint32_t TMEM_COLS = 256;          // two S^T buffers of 128 columns
+  static constexpr int THREADS = kMassThreads;
+  static constexpr int PRODUCER = 4 * NWG, MMA = 4 * NWG + 1;   // warp roles after the mass warpgroups
+  static constexpr uint32_t TMEM_COLS = NWG <= 2 ? 256 : 512;   // NWG S^T buffers of 128 columns
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, 128, 0, 0);
 };
 
@@ -91,8 +95,8 @@ struct MassParams {
 struct MassShared {
   uint64_t item_full[2], item_empty[2];
   uint64_t k_full, k_ready, k_empty;
-  uint64_t q_full[4], q_empty[4];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t q_full[8], q_empty[8];
+  uint64_t s_full[4], s_empty[4];
   uint64_t drain;
   __align__(16) int32_t item[2][M_NFIELDS];
   uint32_t tmem_base;
@@ -100,11 +104,11 @@ struct MassShared {
 };
 
 template <int D, int P>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kMassThreads, 1)
     segpaged_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const MassParams p) {
   using C = MassCfg<D, P>;
-  static_assert(C::NQ <= 4, "barrier arrays hold four query slots");
+  static_assert(C::NQ <= 8 && C::NWG <= 4, "barrier arrays hold eight query slots and four buffers");
   extern __shared__ uint8_t smem_raw[];
   __shared__ MassShared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -118,7 +122,9 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sh.item_full[i], 1);
-      ptx::mbar_init(&sh.item_empty[i], 9);   // MMA warp + 8 mass warps
+      ptx::mbar_init(&sh.item_empty[i], 1 + 4 * C::NWG);   // MMA warp + every mass warp
+    }
+    for (int i = 0; i < C::NWG; ++i) {
       ptx::mbar_init(&sh.s_full[i], 1);
       ptx::mbar_init(&sh.s_empty[i], 4);      // the 4 warps of the buffer's warpgroup
     }
@@ -133,11 +139,11 @@ __global__ void __launch_bounds__(320, 1)
     sh.abort = 0;
     ptx::mbar_fence_init();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == C::PRODUCER && lane == 0) {
     ptx::tma_prefetch_desc(&tm_q);
     ptx::tma_prefetch_desc(&tm_k);
   }
-  if (warp == 9) {
+  if (warp == C::MMA) {
     ptx::tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(320, 1)
   const int G = 1 << p.log2_group;
   const int npos = 128 >> p.log2_group;
 
-  if (warp == 8) {
+  if (warp == C::PRODUCER) {
     // ------------------------------------------------------------------------------ producer
     uint32_t qi = 0, q_issued = 0;
     int32_t k_ring = -1;
@@ -278,7 +284,7 @@ __global__ void __launch_bounds__(320, 1)
         ptx::mbar_wait(&sh.q_full[it % C::NQ], (it / C::NQ) & 1, nullptr, status, kMassStatusTimeout);
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == C::MMA) {
     // --------------------------------------------------------------------------- MMA issuer
     const uint32_t leader = ptx::elect_one();
     const uint32_t k_base = ptx::smem_addr(sK), q_base = ptx::smem_addr(sQ);
@@ -297,8 +303,8 @@ __global__ void __launch_bounds__(320, 1)
       if (nt < 0) break;
       if (!wait(&sh.k_ready, ring & 1)) break;
       for (int32_t t = 0; t < nt; ++t, ++qi, ++si) {
-        const int s = qi % C::NQ, b = si & 1;
-        if (!wait(&sh.q_full[s], (qi / C::NQ) & 1) || !wait(&sh.s_empty[b], ((si >> 1) & 1) ^ 1)) {
+        const int s = qi % C::NQ, b = si % C::NWG;
+        if (!wait(&sh.q_full[s], (qi / C::NQ) & 1) || !wait(&sh.s_empty[b], ((si / C::NWG) & 1) ^ 1)) {
           ok = false;
           break;
         }
@@ -321,7 +327,7 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ----------------------------------------------------------------------- mass warpgroups
-    const int wg = warp >> 2;                            // takes the tiles g with g % 2 == wg
+    const int wg = warp >> 2;                            // takes the tiles g with g % NWG == wg
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;                 // key row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -347,9 +353,9 @@ __global__ void __launch_bounds__(320, 1)
       float sum = 0.f;
       bool ok = true;
       for (int32_t t = 0; t < nt; ++t, ++qi, ++si) {
-        const int s = qi % C::NQ, b = si & 1;
+        const int s = qi % C::NQ, b = si % C::NWG;
         if (b != wg) continue;
-        if (!wwait(&sh.s_full[b], (si >> 1) & 1) || !wwait(&sh.q_full[s], (qi / C::NQ) & 1)) {
+        if (!wwait(&sh.s_full[b], (si / C::NWG) & 1) || !wwait(&sh.q_full[s], (qi / C::NQ) & 1)) {
           ok = false;
           break;
         }
@@ -418,7 +424,7 @@ __global__ void __launch_bounds__(320, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == C::MMA) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }

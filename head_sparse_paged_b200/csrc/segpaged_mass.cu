@@ -88,7 +88,8 @@ extern "C" int64_t segpaged_mass_plan(const segpaged_dims* dims, const int32_t* 
 
 extern "C" size_t segpaged_mass_workspace_bytes(const segpaged_dims* dims, int32_t total_q) {
   if (!dims || dims->num_kv_heads < 1 || total_q < 0) return kMassCounterBytes;
-  return kMassCounterBytes + ((2 * (size_t)dims->num_kv_heads * (size_t)total_q * sizeof(float) + 255) & ~(size_t)255);
+  return kMassCounterBytes +
+         ((kMassWarpgroups * (size_t)dims->num_kv_heads * (size_t)total_q * sizeof(float) + 255) & ~(size_t)255);
 }
 
 namespace {
@@ -174,11 +175,12 @@ extern "C" int segpaged_token_mass(const segpaged_dims* dims, const void* q, int
     if (rc != SEGPAGED_OK) return rc;
   } else {
     // no items: every partial is zero
-    if (cudaMemsetAsync(part, 0, 2 * (size_t)dims->num_kv_heads * total_q * sizeof(float), st) != cudaSuccess)
+    if (cudaMemsetAsync(part, 0, kMassWarpgroups * (size_t)dims->num_kv_heads * total_q * sizeof(float), st) !=
+        cudaSuccess)
       return SEGPAGED_ERR_CUDA;
   }
   const int blocks = (int)std::min<int64_t>((total_q + 255) / 256, (int64_t)sms * 8);
-  mass_reduce_kernel<<<blocks, 256, 0, st>>>(part, mass, total_q, 2 * dims->num_kv_heads);
+  mass_reduce_kernel<<<blocks, 256, 0, st>>>(part, mass, total_q, kMassWarpgroups * dims->num_kv_heads);
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
 }
 

@@ -309,7 +309,7 @@ int64_t segpaged_mass_plan(const segpaged_dims* dims, const int32_t* ctx_len, co
                            const segpaged_head_class* cls, const int32_t* page_table_offs,
                            segpaged_mass_item* items, int64_t capacity);
 
-/* Device workspace segpaged_token_mass needs: two partial sums per (KV head, query row) and a counter. */
+/* Device workspace segpaged_token_mass needs: a few partial sums per (KV head, query row) and a counter. */
 size_t segpaged_mass_workspace_bytes(const segpaged_dims* dims, int32_t total_q);
 
 /*
