@@ -96,7 +96,7 @@ struct PrefillParams {
   __nv_bfloat16* v_pool;
 };
 
-constexpr int kRopeSmemFragments = 256;   // fragment starts of a sequence cached in shared memory
+constexpr int kRopeSmemFragments = 64;    // fragment starts of a sequence cached in shared memory
 
 template <bool ROPE>
 struct PrefillShared {
@@ -108,6 +108,8 @@ struct PrefillShared {
   uint64_t k_rot[10];      // ROPE: K tile of tile count n rotated (ring over n % NSLOT), ready for the MMA
   __align__(16) int32_t unit[2][U_NFIELDS];
   int32_t frag_start[ROPE ? kRopeSmemFragments : 1];   // ROPE: the current unit's sequence fragment starts
+  float ml[256];              // shared half units: warpgroup 1's running max and sum per row, for the merge
+  uint64_t ml_full, ml_empty; // ... written by warpgroup 1 (4 warps), read by warpgroup 0 (4 warps)
   uint32_t tmem_base;
   int abort;
 };
@@ -124,12 +126,16 @@ __device__ __forceinline__ int32_t unit_logical_page(const int32_t* u, int32_t i
 // Kernel variants: the plain prefill, gather-time RoPE, and fused append-and-attend.
 constexpr int kModePlain = 0, kModeRope = 1, kModeAppend = 2;
 
-template <int D, int P, int MODE>
+template <int D, int P, int MODE, bool SHARED_HALF>
 __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
                             const __grid_constant__ CUtensorMap tm_vn, const PrefillParams p) {
   constexpr bool ROPE = MODE == kModeRope, APPEND = MODE == kModeAppend;
+  // SHARED_HALF (chosen per launch: the plan has half units): a unit with rows in one query tile only
+  // still keeps both softmax warpgroups busy -- its KV tiles alternate between them (S buffer, P, O
+  // accumulator t = tile & 1) and warpgroup 0 merges the two accumulators at the end. The variant without
+  // it keeps the long-unit path free of the extra bookkeeping (about 3 % on long layers).
   using C = PrefillCfg<D, P, ROPE>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ PrefillShared<ROPE> sh;
@@ -155,6 +161,8 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     ptx::mbar_init(&sh.q_full, 1);
     ptx::mbar_init(&sh.q_empty, 1);
     ptx::mbar_init(&sh.mma_drain, 1);
+    ptx::mbar_init(&sh.ml_full, 4);
+    ptx::mbar_init(&sh.ml_empty, 4);
     for (int i = 0; i < C::NSLOT; ++i) {
       ptx::mbar_init(&sh.kv_full[i], 1);
       ptx::mbar_init(&sh.kv_empty[i], 1);
@@ -338,11 +346,11 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       };
       // O_t (+)= P_t V for the V tile in KV item vi; `first` starts the unit's accumulation. The softmax
       // warps publish P_t in two halves of 64 keys: the first half's MMAs run while they finish the second.
-      auto issue_pv = [&](int t, uint32_t vi, bool first) -> bool {
+      auto issue_pv = [&](int t, uint32_t vi, bool first, bool wait_v) -> bool {
         if (!wait(&sh.p_half[t], pcount[t] & 1)) return false;
         if (first && act[t] > 0 && !wait(&sh.o_free[t], (act[t] - 1) & 1)) return false;
         const int s = vi % C::NSLOT;
-        if (t == 0 && !wait(&sh.kv_full[s], (vi / C::NSLOT) & 1)) return false;
+        if (wait_v && !wait(&sh.kv_full[s], (vi / C::NSLOT) & 1)) return false;
         ptx::tc_fence_after();
         const uint32_t pa = tmem + t * 128;                 // P_t: bf16 pairs over the first 64 columns of S_t
         const uint32_t od = tmem + 256 + t * D;
@@ -359,9 +367,9 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
           ptx::umma_ts(leader, od, pa + kk * 8, vdesc + (uint64_t)(kk * 128), C::IDESC_O, 1u);
         return true;
       };
-      auto issue_s = [&](int t, uint32_t kb) {
+      auto issue_s = [&](int t, uint32_t kb, int qt) {
         const uint32_t sd = tmem + t * 128;
-        const uint64_t qdesc = ptx::sw128_desc(q_base + t * C::Q_BYTES, 16, 1024);
+        const uint64_t qdesc = ptx::sw128_desc(q_base + qt * C::Q_BYTES, 16, 1024);
         const uint64_t kdesc = ptx::sw128_desc(kb, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -379,35 +387,69 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
         if (ntiles < 0) break;
         if (!wait(&sh.q_full, (ring & 1))) { ok = false; break; }
+        // K of tile j released to the MMA: by the RoPE warps with ROPE (their barrier ring counts K tiles only:
+        // a slot hosts K and V items alike, so the slot's own phase count does not apply), else by the TMA
+        auto k_ready = [&](uint32_t ki) -> bool {
+          return ROPE ? wait(&sh.k_rot[(ki >> 1) % C::NSLOT], ((ki >> 1) / C::NSLOT) & 1)
+                      : wait(&sh.kv_full[ki % C::NSLOT], (ki / C::NSLOT) & 1);
+        };
+        if (SHARED_HALF && !two) {
+          // half unit: tile j uses S buffer, P and O accumulator t = j & 1 over query tile 0; S_t(j) may be
+          // issued once PV_t(j - 2) has been
+          uint32_t v_of[2] = {0, 0};
+          for (int32_t j = 0; j < ntiles && ok; ++j) {
+            const int t = j & 1;
+            const uint32_t ki = kv_item, vi = kv_item + 1;
+            kv_item += 2;
+            if (j >= 2) {
+              if (!issue_pv(t, v_of[t], j < 4, true)) { ok = false; break; }
+              ptx::umma_commit(leader, &sh.kv_empty[v_of[t] % C::NSLOT]);
+            }
+            if (!k_ready(ki)) { ok = false; break; }
+            ptx::tc_fence_after();
+            issue_s(t, kv_base + (ki % C::NSLOT) * C::TILE_BYTES, 0);
+            ptx::umma_commit(leader, &sh.kv_empty[ki % C::NSLOT]);
+            if (j == ntiles - 1) ptx::umma_commit(leader, &sh.q_empty);
+            v_of[t] = vi;
+          }
+          if (!ok) break;
+          // the last PV into each accumulator publishes it
+          for (int32_t j = ntiles >= 2 ? ntiles - 2 : 0; j < ntiles; ++j) {
+            const int t = j & 1;
+            if (!issue_pv(t, v_of[t], j < 2, true)) { ok = false; break; }
+            ptx::umma_commit(leader, &sh.o_full[t]);
+            ptx::umma_commit(leader, &sh.kv_empty[v_of[t] % C::NSLOT]);
+          }
+          if (!ok) break;
+          ++act[0];
+          if (ntiles >= 2) ++act[1];
+          continue;
+        }
         uint32_t prev_vi = 0;
         for (int32_t j = 0; j < ntiles && ok; ++j) {
           const uint32_t ki = kv_item, vi = kv_item + 1;
           kv_item += 2;
-          if (j > 0 && !issue_pv(0, prev_vi, j == 1)) { ok = false; break; }
+          if (j > 0 && !issue_pv(0, prev_vi, j == 1, true)) { ok = false; break; }
           const int s = ki % C::NSLOT;
-          // with ROPE the K tile is released by the RoPE warps; their barrier ring counts K tiles only (a
-          // slot hosts K and V items alike, so the slot's own phase count does not apply)
-          const bool kready = ROPE ? wait(&sh.k_rot[(ki >> 1) % C::NSLOT], ((ki >> 1) / C::NSLOT) & 1)
-                                   : wait(&sh.kv_full[s], (ki / C::NSLOT) & 1);
-          if (!kready) { ok = false; break; }
+          if (!k_ready(ki)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t kb = kv_base + s * C::TILE_BYTES;
-          issue_s(0, kb);
+          issue_s(0, kb, 0);
           if (j > 0) {
-            if (two && !issue_pv(1, prev_vi, j == 1)) { ok = false; break; }
+            if (two && !issue_pv(1, prev_vi, j == 1, false)) { ok = false; break; }
             ptx::umma_commit(leader, &sh.kv_empty[prev_vi % C::NSLOT]);
           }
-          if (two) issue_s(1, kb);
+          if (two) issue_s(1, kb, 1);
           ptx::umma_commit(leader, &sh.kv_empty[s]);
           if (j == ntiles - 1) ptx::umma_commit(leader, &sh.q_empty);
           prev_vi = vi;
         }
         if (!ok) break;
         // the unit's last PV of each tile publishes its O
-        if (!issue_pv(0, prev_vi, ntiles == 1)) break;
+        if (!issue_pv(0, prev_vi, ntiles == 1, true)) break;
         ptx::umma_commit(leader, &sh.o_full[0]);
         if (two) {
-          if (!issue_pv(1, prev_vi, ntiles == 1)) break;
+          if (!issue_pv(1, prev_vi, ntiles == 1, false)) break;
           ptx::umma_commit(leader, &sh.o_full[1]);
         }
         ptx::umma_commit(leader, &sh.kv_empty[prev_vi % C::NSLOT]);
@@ -564,7 +606,10 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     const uint32_t obuf = tmem + 256 + tile * D + lane_off;
     const float sl2 = p.scale_log2;
     const uint64_t sl2_2 = f2_pack(sl2, sl2);
-    uint32_t scount = 0, ucnt = 0;
+    uint32_t scount = 0;
+    // completed uses of O0 and O1 (phases of o_full[0], o_full[1]) and of the half-unit hand-off, counted
+    // by both warpgroups over every unit
+    uint32_t o0cnt = 0, o1cnt = 0, mlcnt = 0;
     // The tcgen05.ld/st below are warp-collective, so every wait's outcome is made warp-uniform.
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kStatusTimeout));
@@ -576,14 +621,16 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       // the epilogue, and the producer refills a slot only once every consumer has released it.
       const int32_t* u = sh.unit[slot];
       const int32_t ntiles = u[U_NTILES];
-      if (ntiles < 0 || (tile == 1 && u[U_HALF])) {   // end of schedule, or no rows for this tile
+      const bool shared_half = SHARED_HALF && u[U_HALF] != 0;   // both warpgroups on query tile 0
+      const bool two_o = shared_half && ntiles >= 2;             // ... and O1 holds warpgroup 1's share
+      if (ntiles < 0 || (tile == 1 && u[U_HALF] && !SHARED_HALF)) {   // end of schedule, or no rows for us
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
         if (ntiles < 0) break;
         continue;
       }
       const int32_t t0 = u[U_T0];
-      const int32_t pslot = tile * npos + (row >> p.log2_group);
+      const int32_t pslot = (shared_half ? 0 : tile) * npos + (row >> p.log2_group);
       const bool valid_row = pslot < u[U_NPOS];
       const int32_t i_pos = u[U_POS0] + (valid_row ? pslot : u[U_NPOS] - 1);
       const int32_t head = u[U_KVH] * G + (row & (G - 1));
@@ -595,7 +642,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
 
-      for (int32_t j = 0; j < ntiles; ++j) {
+      for (int32_t j = shared_half ? tile : 0; j < ntiles; j += shared_half ? 2 : 1) {
         // Logical page of every slot of this KV tile, worked out before S is ready; a row needs per-column
         // bounds only if some key of the tile is invisible to it (causal edge, window edge, sink tail, a
         // short last tile, or -- appending -- the page holding q0, split between pool and new K/V).
@@ -735,8 +782,64 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       if (!ok) break;
 
       // ------------------------------------------------------------------------------ epilogue
-      if (!wwait(&sh.o_full[tile], ucnt & 1)) break;
+      if (shared_half && tile == 1) {
+        // hand the running max and sum of warpgroup 1's KV tiles to warpgroup 0, which merges
+        if (two_o) {
+          // the previous hand-off has been read
+          if (!wwait(&sh.ml_empty, (mlcnt & 1) ^ 1)) break;
+          sh.ml[2 * row] = m_run;
+          sh.ml[2 * row + 1] = l_run;
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&sh.ml_full);
+          ++o1cnt;
+          ++mlcnt;
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
+        continue;
+      }
+      if (!wwait(&sh.o_full[tile], (tile == 0 ? o0cnt : o1cnt) & 1)) break;
+      // weights of the two accumulators: (1, 0) unless this is a shared half unit with two shares
+      float a0 = 1.f, a1 = 0.f;
+      if (two_o) {
+        if (!wwait(&sh.ml_full, mlcnt & 1) || !wwait(&sh.o_full[1], o1cnt & 1)) break;
+        const float m1 = sh.ml[2 * row], l1 = sh.ml[2 * row + 1];
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.ml_empty);
+        const float M = fmaxf(m_run, m1);
+        a0 = (m_run == -INFINITY) ? 0.f : ptx::ex2(m_run - M);
+        a1 = (m1 == -INFINITY) ? 0.f : ptx::ex2(m1 - M);
+        l_run = a0 * l_run + a1 * l1;
+        m_run = M;
+      }
+      const uint32_t obuf1 = tmem + 256 + D + lane_off;   // O1, merged into O0's rows
       ptx::tc_fence_after();
+      // O chunk c of this warpgroup's rows, merged with O1 for a shared half unit
+      auto load_o = [&](int c, uint32_t (&r)[32]) {
+        ptx::tmem_ld32(obuf + c * 32, r);
+        if (two_o) {
+          uint32_t r1[32];
+          ptx::tmem_ld32(obuf1 + c * 32, r1);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            r[k] = __float_as_uint(__fmaf_rn(a1, __uint_as_float(r1[k]), a0 * __uint_as_float(r[k])));
+        } else {
+          ptx::tmem_ld_wait();
+        }
+      };
+      auto release = [&] {
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(&sh.o_free[tile]);
+          if (two_o) ptx::mbar_arrive(&sh.o_free[1]);   // warpgroup 0 read O1 too
+          ptx::mbar_arrive(&sh.unit_empty[slot]);
+        }
+        ++o0cnt;                                   // every unit publishes O0
+        if (!u[U_HALF] || two_o) ++o1cnt;          // full units and shared half units with two shares, O1
+        if (two_o) ++mlcnt;
+      };
       const int32_t part = u[U_PART];
       if (part >= 0) {
         // one chunk of a split unit: O / l in fp32 and the chunk's LSE, for the combine pass; a row that
@@ -748,8 +851,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
-          ptx::tmem_ld32(obuf + c * 32, r);
-          ptx::tmem_ld_wait();
+          load_o(c, r);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             reinterpret_cast<float4*>(dst + c * 32)[k] =
@@ -757,13 +859,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
                             __uint_as_float(r[4 * k + 2]) * inv_l, __uint_as_float(r[4 * k + 3]) * inv_l);
         }
         p.part_lse[prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(&sh.o_free[tile]);
-          ptx::mbar_arrive(&sh.unit_empty[slot]);
-        }
-        ++ucnt;
+        release();
         continue;
       }
       const float inv_l = 1.0f / l_run;
@@ -772,8 +868,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        ptx::tmem_ld32(obuf + c * 32, r);
-        ptx::tmem_ld_wait();
+        load_o(c, r);
         uint32_t w[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
@@ -785,13 +880,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         }
       }
       if (valid_row) p.lse[(int64_t)head * p.total_q + qrow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive(&sh.o_free[tile]);
-        ptx::mbar_arrive(&sh.unit_empty[slot]);
-      }
-      ++ucnt;
+      release();
     }
   }
 

@@ -314,6 +314,8 @@ int64_t plan_units(const segpaged_dims* dims, const int32_t* ctx_len, const int3
     info->num_units = (int64_t)out.size();
     info->num_groups = (int64_t)groups.size();
     info->num_partials = slots;
+    info->num_half_units = 0;
+    for (const auto& u : out) info->num_half_units += u.v[U_HALF] ? 1 : 0;
   }
   out.insert(out.end(), groups.begin(), groups.end());
   const int64_t n = (int64_t)out.size();
@@ -390,21 +392,29 @@ size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpage
 
 namespace {
 
-template <int D, int P, int MODE>
-int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkn,
-                   const CUtensorMap& tvn, const PrefillParams& p, int grid, cudaStream_t st) {
+template <int D, int P, int MODE, bool HALF>
+int launch_prefill_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkn,
+                     const CUtensorMap& tvn, const PrefillParams& p, int grid, cudaStream_t st) {
   using C = PrefillCfg<D, P, MODE == kModeRope>;
   static bool configured[kMaxDevices] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(segpaged_prefill_kernel<D, P, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(segpaged_prefill_kernel<D, P, MODE, HALF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return SEGPAGED_ERR_CUDA;
     configured[dev] = true;
   }
-  segpaged_prefill_kernel<D, P, MODE><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tkn, tvn, p);
+  segpaged_prefill_kernel<D, P, MODE, HALF><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tkn, tvn, p);
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
+}
+
+// The shared-half variant when the plan has half units (rows in one query tile only).
+template <int D, int P, int MODE>
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkn,
+                   const CUtensorMap& tvn, const PrefillParams& p, int grid, cudaStream_t st, bool half) {
+  return half ? launch_prefill_v<D, P, MODE, true>(tq, tk, tv, tkn, tvn, p, grid, st)
+              : launch_prefill_v<D, P, MODE, false>(tq, tk, tv, tkn, tvn, p, grid, st);
 }
 
 }  // namespace
@@ -490,6 +500,7 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   p.log2_group = log2_int(G);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.frags = frags ? *frags : RopeFragments{nullptr, nullptr, nullptr};
+  const bool half = info->num_half_units > 0;
   p.append = append ? 1 : 0;
   p.num_kv_heads = dims->num_kv_heads;
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
@@ -500,9 +511,9 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   rc = SEGPAGED_ERR_DIMS;
 #define SEGPAGED_LAUNCH(DD, PP)                                                   \
   if (D == DD && P == PP)                                                          \
-    rc = frags    ? launch_prefill<DD, PP, kModeRope>(tq, tk, tv, tkn, tvn, p, grid, st)   \
-         : append ? launch_prefill<DD, PP, kModeAppend>(tq, tk, tv, tkn, tvn, p, grid, st) \
-                  : launch_prefill<DD, PP, kModePlain>(tq, tk, tv, tkn, tvn, p, grid, st);
+    rc = frags    ? launch_prefill<DD, PP, kModeRope>(tq, tk, tv, tkn, tvn, p, grid, st, half)   \
+         : append ? launch_prefill<DD, PP, kModeAppend>(tq, tk, tv, tkn, tvn, p, grid, st, half) \
+                  : launch_prefill<DD, PP, kModePlain>(tq, tk, tv, tkn, tvn, p, grid, st, half);
   SEGPAGED_LAUNCH(128, 16)
   SEGPAGED_LAUNCH(128, 32)
   SEGPAGED_LAUNCH(128, 64)
@@ -624,6 +635,8 @@ extern "C" int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const vo
   info.num_units = num_units;
   info.num_groups = 0;
   info.num_partials = 0;
+  info.num_half_units = 0;
+  for (int64_t i = 0; i < num_units; ++i) info.num_half_units += units_host[i].v[U_HALF] ? 1 : 0;
   return segpaged_attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len,
                                reinterpret_cast<const segpaged_unit*>(units_dev), &info, softmax_scale, o, lse,
                                scratch, kNoAllocUnitOffset * sizeof(int32_t), status, stream);

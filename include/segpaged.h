@@ -90,11 +90,15 @@ typedef struct {
 } segpaged_unit;
 
 /* Shape of a plan: records [0, num_units) are work units, records [num_units, num_units + num_groups)
- * combine records; num_partials partial-result slots live in the workspace. */
+ * combine records; num_partials partial-result slots live in the workspace; num_half_units of the units
+ * have rows in one query tile only. num_half_units only picks a kernel variant (> 0: each such unit's KV
+ * tiles alternate between both softmax warpgroups, which merge their two partial results at the end);
+ * results are correct for any value, but the two variants round differently. */
 typedef struct {
   int64_t num_units;
   int64_t num_groups;
   int64_t num_partials;
+  int64_t num_half_units;
 } segpaged_plan_info;
 
 /* Text for an error code (static storage). */
