@@ -17,6 +17,18 @@
 namespace segpaged {
 
 constexpr int kCombineMaxSplit = 256;  // chunks per unit (the planner never makes more)
+constexpr int kCombineWideSplit = 16;  // records with more chunks get a block per row, the others a warp
+constexpr int kCombineRows = 256;      // rows of a combine record (two query tiles)
+constexpr int32_t kCombineStatusUnit = 8;   // SEGPAGED_STATUS_UNIT: the grid had too few row blocks
+
+// Thread blocks the combine launch needs for one record: up to its last valid row (a query tile holds
+// 128/G positions x G heads, the second tile from row 128), one block per row for a wide record, one per
+// 8 rows otherwise.
+SP_HD int64_t combine_blocks_of(int32_t npos, int32_t nsplit, int32_t G) {
+  const int32_t npos_tile = 128 / G;
+  const int32_t rows = npos <= npos_tile ? npos * G : 128 + (npos - npos_tile) * G;
+  return nsplit > kCombineWideSplit ? rows : ceil_div(rows, 8);
+}
 
 struct CombineParams {
   const int32_t* records;  // combine records [num_groups][U_NFIELDS]
@@ -26,6 +38,8 @@ struct CombineParams {
   __nv_bfloat16* o;        // [total_q, Hq, D]
   float* lse;              // [Hq, total_q]
   int32_t total_q, num_q_heads, log2_group;
+  int32_t row_blocks;      // gridDim.y: the most row blocks a record needs
+  int32_t* status;         // nullable
 };
 
 // Online merge of chunks c = c0, c0 + stride, ... into (m, wsum, acc): loads of four chunks are issued
@@ -71,9 +85,10 @@ __device__ __forceinline__ void merge_chunks(const float* part_o, const float* p
   }
 }
 
-// grid: (combine records, 256). A record with at most 16 chunks gets one warp per row (blockIdx.y picks a
-// block of 8 rows); a wider record gets all 8 warps of a block on one row (blockIdx.y is the row), warp w
-// merging chunks c = w (mod 8), and the eight partial triples are merged in order 0..7.
+// grid: (combine records, row blocks: as many as the widest record needs, at most 256). A record with at
+// most 16 chunks gets one warp per row (blockIdx.y picks a block of 8 rows); a wider record gets all 8
+// warps of a block on one row (blockIdx.y is the row), warp w merging chunks c = w (mod 8), and the eight
+// partial triples are merged in order 0..7.
 template <int D>
 __global__ void __launch_bounds__(256) segpaged_combine_kernel(const CombineParams p) {
   constexpr int V = D / 32;  // columns per lane
@@ -91,7 +106,11 @@ __global__ void __launch_bounds__(256) segpaged_combine_kernel(const CombinePara
     const int32_t part0 = rec[U_PART], nsplit = rec[U_NSPLIT], npos = rec[U_NPOS];
     const int32_t qrow0 = rec[U_QROW], kvh = rec[U_KVH];
     const int rows = rec[U_HALF] ? 128 : 256;
-    const bool wide = nsplit > 16;
+    const bool wide = nsplit > kCombineWideSplit;
+    // the last row block checks that the grid reaches every valid row of the record
+    if (blockIdx.y == gridDim.y - 1 && threadIdx.x == 0 && p.status &&
+        combine_blocks_of(npos, nsplit, G) > (int64_t)gridDim.y)
+      atomicOr(p.status, kCombineStatusUnit);
     const int r = wide ? (int)blockIdx.y : (int)blockIdx.y * NW + warp;
     if ((wide ? r : (int)blockIdx.y * NW) >= rows) continue;     // uniform for the whole block
     const int tile = r >> 7, rr = r & 127;

@@ -104,8 +104,8 @@ struct PrefillShared {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_half[2], p_full[2], o_full[2], o_free[2];
   uint64_t mma_drain;
-  uint64_t kv_full[10], kv_empty[10];
-  uint64_t k_rot[10];      // ROPE: K tile of tile count n rotated (ring over n % NSLOT), ready for the MMA
+  uint64_t kv_full[11], kv_empty[11];
+  uint64_t k_rot[11];      // ROPE: K tile of tile count n rotated (ring over n % NSLOT), ready for the MMA
   __align__(16) int32_t unit[2][U_NFIELDS];
   int32_t frag_start[ROPE ? kRopeSmemFragments : 1];   // ROPE: the current unit's sequence fragment starts
   float ml[256];              // shared half units: warpgroup 1's running max and sum per row, for the merge
@@ -126,22 +126,30 @@ __device__ __forceinline__ int32_t unit_logical_page(const int32_t* u, int32_t i
 // Kernel variants: the plain prefill, gather-time RoPE, and fused append-and-attend.
 constexpr int kModePlain = 0, kModeRope = 1, kModeAppend = 2;
 
-template <int D, int P, int MODE, bool SHARED_HALF>
+// HALF (chosen per launch): 0 -- every unit has rows in both query tiles; 1 -- the plan has half units;
+// 2 -- every unit is a half unit.
+template <int D, int P, int MODE, int HALF>
 __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
                             const __grid_constant__ CUtensorMap tm_vn, const PrefillParams p) {
   constexpr bool ROPE = MODE == kModeRope, APPEND = MODE == kModeAppend;
-  // SHARED_HALF (chosen per launch: the plan has half units): a unit with rows in one query tile only
-  // still keeps both softmax warpgroups busy -- its KV tiles alternate between them (S buffer, P, O
-  // accumulator t = tile & 1) and warpgroup 0 merges the two accumulators at the end. The variant without
-  // it keeps the long-unit path free of the extra bookkeeping (about 3 % on long layers).
+  // SHARED_HALF (the plan has half units): a unit with rows in one query tile only still keeps both softmax
+  // warpgroups busy -- its KV tiles alternate between them (S buffer, P, O accumulator t = tile & 1) and
+  // warpgroup 0 merges the two accumulators at the end. The variant without it keeps the long-unit path
+  // free of the extra bookkeeping (about 3 % on long layers).
+  // ALL_HALF (every unit is a half unit -- short query ranges, decode-like batches): the second query
+  // buffer is never loaded, so it becomes one more K/V slot; these launches stream pages and are bound by
+  // how many loads each SM keeps in flight.
+  constexpr bool SHARED_HALF = HALF != 0, ALL_HALF = HALF == 2;
   using C = PrefillCfg<D, P, ROPE>;
+  constexpr int NSLOT = C::NSLOT + (ALL_HALF ? 1 : 0);   // K/V slots of this variant
+  static_assert(C::Q_BYTES == C::TILE_BYTES, "a query buffer doubles as a K/V slot");
   extern __shared__ uint8_t smem_raw[];
   __shared__ PrefillShared<ROPE> sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                        // 2 query tiles x Q_BYTES
-  uint8_t* sKV = smem + 2 * C::Q_BYTES;      // NSLOT x TILE_BYTES
+  uint8_t* sQ = smem;                                      // 2 query tiles x Q_BYTES (1 with ALL_HALF)
+  uint8_t* sKV = smem + (ALL_HALF ? 1 : 2) * C::Q_BYTES;   // NSLOT x TILE_BYTES
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &sh.abort;
   int32_t* status = p.status;
@@ -163,7 +171,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     ptx::mbar_init(&sh.mma_drain, 1);
     ptx::mbar_init(&sh.ml_full, 4);
     ptx::mbar_init(&sh.ml_empty, 4);
-    for (int i = 0; i < C::NSLOT; ++i) {
+    for (int i = 0; i < NSLOT; ++i) {
       ptx::mbar_init(&sh.kv_full[i], 1);
       ptx::mbar_init(&sh.kv_empty[i], 1);
       ptx::mbar_init(&sh.k_rot[i], 4);
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
   // rows it does not load, and those columns are masked. With one page per tile every used slot is loaded
   // whole, and the start-up saves the stores.
   if constexpr (C::PPT > 1) {
-    for (int x = threadIdx.x; x < C::NSLOT * C::TILE_BYTES / 16; x += blockDim.x)
+    for (int x = threadIdx.x; x < NSLOT * C::TILE_BYTES / 16; x += blockDim.x)
       reinterpret_cast<uint4*>(sKV)[x] = make_uint4(0, 0, 0, 0);
   }
   // The combine launch that may follow this one (split plans) can be scheduled as SMs free up; it waits
@@ -235,7 +243,10 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         if (lane == 0) {
           go = ptx::mbar_wait(&sh.q_empty, (ring & 1) ^ 1, abort, status, kStatusTimeout);
           if (go) {
-            const int nq = U[U_HALF] ? 1 : 2;   // a half unit has no rows in its second query tile
+            // a half unit has no rows in its second query tile; with ALL_HALF a unit that is not half is a
+            // plan that does not match the launch, and only its first query tile is computed
+            if (ALL_HALF && !U[U_HALF] && status) atomicOr(status, kStatusUnit);
+            const int nq = (ALL_HALF || U[U_HALF]) ? 1 : 2;
             ptx::mbar_arrive_expect_tx(&sh.q_full, nq * C::Q_BYTES);
             q_ring = (int32_t)ring;
             for (int t = 0; t < nq; ++t)
@@ -296,8 +307,8 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
 #pragma unroll
             for (int which = 0; which < 2; ++which) {  // K then V
               const uint32_t item = kv_item + which;
-              const int s = item % C::NSLOT;
-              if (!ptx::mbar_wait(&sh.kv_empty[s], ((item / C::NSLOT) & 1) ^ 1, abort, status, kStatusTimeout)) {
+              const int s = item % NSLOT;
+              if (!ptx::mbar_wait(&sh.kv_empty[s], ((item / NSLOT) & 1) ^ 1, abort, status, kStatusTimeout)) {
                 ok = 0;
                 break;
               }
@@ -327,9 +338,9 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       // After giving up, wait (bounded, ignoring the abort flag) for the copies this warp issued, so
       // none lands in shared memory after the CTA has exited.
       if (lane == 0 && *abort) {
-        const uint32_t first = kv_issued > (uint32_t)C::NSLOT ? kv_issued - C::NSLOT : 0u;
+        const uint32_t first = kv_issued > (uint32_t)NSLOT ? kv_issued - NSLOT : 0u;
         for (uint32_t it = first; it < kv_issued; ++it)
-          ptx::mbar_wait(&sh.kv_full[it % C::NSLOT], (it / C::NSLOT) & 1, nullptr, status, kStatusTimeout);
+          ptx::mbar_wait(&sh.kv_full[it % NSLOT], (it / NSLOT) & 1, nullptr, status, kStatusTimeout);
         if (q_ring >= 0) ptx::mbar_wait(&sh.q_full, (uint32_t)q_ring & 1, nullptr, status, kStatusTimeout);
       }
       __syncwarp();
@@ -349,8 +360,8 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       auto issue_pv = [&](int t, uint32_t vi, bool first, bool wait_v) -> bool {
         if (!wait(&sh.p_half[t], pcount[t] & 1)) return false;
         if (first && act[t] > 0 && !wait(&sh.o_free[t], (act[t] - 1) & 1)) return false;
-        const int s = vi % C::NSLOT;
-        if (wait_v && !wait(&sh.kv_full[s], (vi / C::NSLOT) & 1)) return false;
+        const int s = vi % NSLOT;
+        if (wait_v && !wait(&sh.kv_full[s], (vi / NSLOT) & 1)) return false;
         ptx::tc_fence_after();
         const uint32_t pa = tmem + t * 128;                 // P_t: bf16 pairs over the first 64 columns of S_t
         const uint32_t od = tmem + 256 + t * D;
@@ -382,7 +393,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         const int slot = ring & 1;
         if (!wait(&sh.unit_full[slot], (ring >> 1) & 1)) { ok = false; break; }
         const int32_t ntiles = sh.unit[slot][U_NTILES];
-        const bool two = sh.unit[slot][U_HALF] == 0;   // second query tile active
+        const bool two = !ALL_HALF && sh.unit[slot][U_HALF] == 0;   // second query tile active
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
         if (ntiles < 0) break;
@@ -390,8 +401,8 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         // K of tile j released to the MMA: by the RoPE warps with ROPE (their barrier ring counts K tiles only:
         // a slot hosts K and V items alike, so the slot's own phase count does not apply), else by the TMA
         auto k_ready = [&](uint32_t ki) -> bool {
-          return ROPE ? wait(&sh.k_rot[(ki >> 1) % C::NSLOT], ((ki >> 1) / C::NSLOT) & 1)
-                      : wait(&sh.kv_full[ki % C::NSLOT], (ki / C::NSLOT) & 1);
+          return ROPE ? wait(&sh.k_rot[(ki >> 1) % NSLOT], ((ki >> 1) / NSLOT) & 1)
+                      : wait(&sh.kv_full[ki % NSLOT], (ki / NSLOT) & 1);
         };
         if (SHARED_HALF && !two) {
           // half unit: tile j uses S buffer, P and O accumulator t = j & 1 over query tile 0; S_t(j) may be
@@ -403,12 +414,12 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
             kv_item += 2;
             if (j >= 2) {
               if (!issue_pv(t, v_of[t], j < 4, true)) { ok = false; break; }
-              ptx::umma_commit(leader, &sh.kv_empty[v_of[t] % C::NSLOT]);
+              ptx::umma_commit(leader, &sh.kv_empty[v_of[t] % NSLOT]);
             }
             if (!k_ready(ki)) { ok = false; break; }
             ptx::tc_fence_after();
-            issue_s(t, kv_base + (ki % C::NSLOT) * C::TILE_BYTES, 0);
-            ptx::umma_commit(leader, &sh.kv_empty[ki % C::NSLOT]);
+            issue_s(t, kv_base + (ki % NSLOT) * C::TILE_BYTES, 0);
+            ptx::umma_commit(leader, &sh.kv_empty[ki % NSLOT]);
             if (j == ntiles - 1) ptx::umma_commit(leader, &sh.q_empty);
             v_of[t] = vi;
           }
@@ -418,7 +429,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
             const int t = j & 1;
             if (!issue_pv(t, v_of[t], j < 2, true)) { ok = false; break; }
             ptx::umma_commit(leader, &sh.o_full[t]);
-            ptx::umma_commit(leader, &sh.kv_empty[v_of[t] % C::NSLOT]);
+            ptx::umma_commit(leader, &sh.kv_empty[v_of[t] % NSLOT]);
           }
           if (!ok) break;
           ++act[0];
@@ -430,14 +441,14 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
           const uint32_t ki = kv_item, vi = kv_item + 1;
           kv_item += 2;
           if (j > 0 && !issue_pv(0, prev_vi, j == 1, true)) { ok = false; break; }
-          const int s = ki % C::NSLOT;
+          const int s = ki % NSLOT;
           if (!k_ready(ki)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t kb = kv_base + s * C::TILE_BYTES;
           issue_s(0, kb, 0);
           if (j > 0) {
             if (two && !issue_pv(1, prev_vi, j == 1, false)) { ok = false; break; }
-            ptx::umma_commit(leader, &sh.kv_empty[prev_vi % C::NSLOT]);
+            ptx::umma_commit(leader, &sh.kv_empty[prev_vi % NSLOT]);
           }
           if (two) issue_s(1, kb, 1);
           ptx::umma_commit(leader, &sh.kv_empty[s]);
@@ -452,7 +463,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
           if (!issue_pv(1, prev_vi, ntiles == 1, false)) break;
           ptx::umma_commit(leader, &sh.o_full[1]);
         }
-        ptx::umma_commit(leader, &sh.kv_empty[prev_vi % C::NSLOT]);
+        ptx::umma_commit(leader, &sh.kv_empty[prev_vi % NSLOT]);
         ++act[0];
         if (two) ++act[1];
       }
@@ -549,8 +560,8 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         for (int32_t j = 0; j < ntiles; ++j) {
           const uint32_t ki = kv_item;
           kv_item += 2;
-          const int s = ki % C::NSLOT;
-          if (!wwait(&sh.kv_full[s], (ki / C::NSLOT) & 1)) { ok = false; break; }
+          const int s = ki % NSLOT;
+          if (!wwait(&sh.kv_full[s], (ki / NSLOT) & 1)) { ok = false; break; }
           if (nfr > 0) {
             uint8_t* tile = sKV + s * C::TILE_BYTES;
             auto token_of = [&](int32_t pos, int r) {
@@ -588,7 +599,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
             ptx::fence_proxy_async_smem();            // the rotated rows are read by the tensor core
           }
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&sh.k_rot[(ki >> 1) % C::NSLOT]);
+          if (lane == 0) ptx::mbar_arrive(&sh.k_rot[(ki >> 1) % NSLOT]);
         }
         if (!ok) break;
         __syncwarp();
@@ -621,9 +632,10 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       // the epilogue, and the producer refills a slot only once every consumer has released it.
       const int32_t* u = sh.unit[slot];
       const int32_t ntiles = u[U_NTILES];
-      const bool shared_half = SHARED_HALF && u[U_HALF] != 0;   // both warpgroups on query tile 0
+      const bool is_half = ALL_HALF || u[U_HALF] != 0;
+      const bool shared_half = SHARED_HALF && is_half;           // both warpgroups on query tile 0
       const bool two_o = shared_half && ntiles >= 2;             // ... and O1 holds warpgroup 1's share
-      if (ntiles < 0 || (tile == 1 && u[U_HALF] && !SHARED_HALF)) {   // end of schedule, or no rows for us
+      if (ntiles < 0 || (tile == 1 && is_half && !SHARED_HALF)) {   // end of schedule, or no rows for us
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
         if (ntiles < 0) break;
@@ -720,7 +732,11 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         const float m_tile = mx * sl2;
         const float m_new = fmaxf(m_run, m_tile);
         bool resc = false;
-        if (j == 0) {
+        if (j == 0 || (SHARED_HALF && m_run == -INFINITY)) {
+          // No visible key of this row so far: O_t holds nothing of it (zeros, or the previous unit's values
+          // that the first P V overwrites), so nothing is rescaled. On a shared half unit this must not touch
+          // O1 at all: warpgroup 1 starts at tile 1 while warpgroup 0 may still be reading the previous
+          // unit's O1 for its merge.
           m_run = m_new;
         } else {
           resc = m_new > m_run + 8.0f;
@@ -837,7 +853,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
           ptx::mbar_arrive(&sh.unit_empty[slot]);
         }
         ++o0cnt;                                   // every unit publishes O0
-        if (!u[U_HALF] || two_o) ++o1cnt;          // full units and shared half units with two shares, O1
+        if (!is_half || two_o) ++o1cnt;            // full units and shared half units with two shares, O1
         if (two_o) ++mlcnt;
       };
       const int32_t part = u[U_PART];

@@ -316,6 +316,10 @@ int64_t plan_units(const segpaged_dims* dims, const int32_t* ctx_len, const int3
     info->num_partials = slots;
     info->num_half_units = 0;
     for (const auto& u : out) info->num_half_units += u.v[U_HALF] ? 1 : 0;
+    info->combine_row_blocks = 0;
+    for (const auto& g : groups)
+      info->combine_row_blocks =
+          std::max(info->combine_row_blocks, combine_blocks_of(g.v[U_NPOS], g.v[U_NSPLIT], G));
   }
   out.insert(out.end(), groups.begin(), groups.end());
   const int64_t n = (int64_t)out.size();
@@ -392,7 +396,7 @@ size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpage
 
 namespace {
 
-template <int D, int P, int MODE, bool HALF>
+template <int D, int P, int MODE, int HALF>
 int launch_prefill_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkn,
                      const CUtensorMap& tvn, const PrefillParams& p, int grid, cudaStream_t st) {
   using C = PrefillCfg<D, P, MODE == kModeRope>;
@@ -409,12 +413,16 @@ int launch_prefill_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;
 }
 
-// The shared-half variant when the plan has half units (rows in one query tile only).
+// The shared-half variant when the plan has half units (rows in one query tile only); for the plain kernel
+// with half units only, the variant that turns the unused second query buffer into one more K/V slot.
 template <int D, int P, int MODE>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkn,
-                   const CUtensorMap& tvn, const PrefillParams& p, int grid, cudaStream_t st, bool half) {
-  return half ? launch_prefill_v<D, P, MODE, true>(tq, tk, tv, tkn, tvn, p, grid, st)
-              : launch_prefill_v<D, P, MODE, false>(tq, tk, tv, tkn, tvn, p, grid, st);
+                   const CUtensorMap& tvn, const PrefillParams& p, int grid, cudaStream_t st, int half) {
+  if constexpr (MODE == kModePlain) {
+    if (half == 2) return launch_prefill_v<D, P, MODE, 2>(tq, tk, tv, tkn, tvn, p, grid, st);
+  }
+  return half ? launch_prefill_v<D, P, MODE, 1>(tq, tk, tv, tkn, tvn, p, grid, st)
+              : launch_prefill_v<D, P, MODE, 0>(tq, tk, tv, tkn, tvn, p, grid, st);
 }
 
 }  // namespace
@@ -422,10 +430,11 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 template <int D>
 int launch_combine(const CombineParams& c, cudaStream_t st) {
   if (c.num_groups <= 0) return SEGPAGED_OK;
-  // records x tile rows, as a programmatic dependent launch: its blocks are scheduled while the prefill's
-  // last CTAs finish and wait in the kernel for that grid's completion
+  // records x row blocks (as many as the widest record needs), as a programmatic dependent launch: its
+  // blocks are scheduled while the prefill's last CTAs finish and wait in the kernel for that grid's
+  // completion
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)std::min<int64_t>(c.num_groups, 65535), 256);
+  cfg.gridDim = dim3((unsigned)std::min<int64_t>(c.num_groups, 65535), (unsigned)c.row_blocks);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
@@ -500,7 +509,8 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   p.log2_group = log2_int(G);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.frags = frags ? *frags : RopeFragments{nullptr, nullptr, nullptr};
-  const bool half = info->num_half_units > 0;
+  // 0: no half units; 1: some; 2: all of them
+  const int half = info->num_half_units <= 0 ? 0 : (info->num_half_units >= num_units ? 2 : 1);
   p.append = append ? 1 : 0;
   p.num_kv_heads = dims->num_kv_heads;
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
@@ -534,6 +544,9 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   c.total_q = total_q;
   c.num_q_heads = Hq;
   c.log2_group = p.log2_group;
+  c.status = status;
+  const int64_t rb = info->combine_row_blocks;
+  c.row_blocks = (rb > 0 && rb < kCombineRows) ? (int32_t)rb : kCombineRows;
   return D == 128 ? launch_combine<128>(c, st) : launch_combine<64>(c, st);
 }
 }  // namespace
@@ -637,6 +650,7 @@ extern "C" int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const vo
   info.num_partials = 0;
   info.num_half_units = 0;
   for (int64_t i = 0; i < num_units; ++i) info.num_half_units += units_host[i].v[U_HALF] ? 1 : 0;
+  info.combine_row_blocks = 0;
   return segpaged_attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len,
                                reinterpret_cast<const segpaged_unit*>(units_dev), &info, softmax_scale, o, lse,
                                scratch, kNoAllocUnitOffset * sizeof(int32_t), status, stream);

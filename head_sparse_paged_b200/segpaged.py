@@ -39,7 +39,7 @@ class SegPagedError(RuntimeError):
 
 class _PlanInfo(ctypes.Structure):
     _fields_ = [("num_units", ctypes.c_int64), ("num_groups", ctypes.c_int64), ("num_partials", ctypes.c_int64),
-                ("num_half_units", ctypes.c_int64)]
+                ("num_half_units", ctypes.c_int64), ("combine_row_blocks", ctypes.c_int64)]
 
 
 class _Dims(ctypes.Structure):
@@ -185,7 +185,8 @@ def segpaged_build(dims: Dims, k_dense, v_dense, cu_seqlens_k, q_len, cls, page_
 
 
 def _info(d: dict) -> _PlanInfo:
-    return _PlanInfo(int(d["num_units"]), int(d["num_groups"]), int(d["num_partials"]), int(d.get("num_half_units", 0)))
+    return _PlanInfo(int(d["num_units"]), int(d["num_groups"]), int(d["num_partials"]), int(d.get("num_half_units", 0)),
+                     int(d.get("combine_row_blocks", 0)))
 
 
 def _plan(fn, name, dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas):
@@ -202,7 +203,7 @@ def _plan(fn, name, dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas
     if n2 < 0:
         raise SegPagedError(int(n2), name)
     return units[:n], {"num_units": info.num_units, "num_groups": info.num_groups, "num_partials": info.num_partials,
-                       "num_half_units": info.num_half_units}
+                       "num_half_units": info.num_half_units, "combine_row_blocks": info.combine_row_blocks}
 
 
 def segpaged_prefill_plan(dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas: int = 0):

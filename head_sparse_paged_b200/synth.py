@@ -128,6 +128,23 @@ def qwen3_32b_small_q(lq: int) -> Workload:
     return w
 
 
+def llama_70b_decode(num_seqs: int = 32, lq: int = 16) -> Workload:
+    """Decode-like batch on Llama-3.3-70B-shaped heads: `num_seqs` sequences with L_b ~ U[16384, 32768], each
+    querying only its last `lq` positions (a multi-token decode or draft-verification step), 64/8 heads, D=128,
+    P=64; per sequence one global KV head at a seeded index, the rest local (S=128, W=2048); pages interleaved
+    across sequences. The stored pages dominate the bytes moved, so the launch is HBM-bound."""
+    rng = np.random.default_rng(1006)
+    L = [int(x) for x in rng.integers(16384, 32769, size=num_seqs)]
+    rows = []
+    for _ in range(num_seqs):
+        g = int(rng.integers(8))
+        rows.append([GLOBAL if k == g else _local(128, 2048) for k in range(8)])
+    return Workload(f"llama-3.3-70b-decode{num_seqs}x{lq}", L, [lq] * num_seqs, 64, 8, 128, 64,
+                    np.array([rows], np.int32), seed=1006, page_order="interleaved",
+                    description=f"Llama-3.3-70B-shaped decode-like batch: {num_seqs} seqs, L~U[16K,32K], Lq={lq}, "
+                                f"Hq=64, Hkv=8, D=128, P=64")
+
+
 def dsv4_flash(layers: int = 43) -> Workload:
     """DeepSeek-V4-Flash-style head split: `layers` layers of 64 MHA heads (own KV each), D=128, one sequence
     L=131072 with Lq=4096, P=128, fully shuffled pool. Layers 0-2 and the last three are all global;
@@ -162,6 +179,7 @@ WORKLOADS = {
     "dsv4-flash": dsv4_flash,
     "qwen3-32b-lq16": lambda: qwen3_32b_small_q(16),
     "qwen3-32b-lq64": lambda: qwen3_32b_small_q(64),
+    "llama-3.3-70b-decode32x16": lambda: llama_70b_decode(32, 16),
 }
 
 

@@ -64,7 +64,8 @@ extern "C" {
 #define SEGPAGED_STATUS_PAGE_ID 1   /* a page id was outside [0, num_pages); it was clamped */
 #define SEGPAGED_STATUS_TABLE 2     /* a head's page-table length disagreed with the storage rule */
 #define SEGPAGED_STATUS_TIMEOUT 4   /* a pipeline wait gave up; outputs of this call are undefined */
-#define SEGPAGED_STATUS_UNIT 8      /* a work unit referenced entries past the page table */
+#define SEGPAGED_STATUS_UNIT 8      /* a plan record did not fit the page table or the call: entries past the
+                                       page table, or a plan that disagrees with its info or entry point */
 
 typedef struct {
   int32_t num_seqs;      /* B */
@@ -92,13 +93,18 @@ typedef struct {
 /* Shape of a plan: records [0, num_units) are work units, records [num_units, num_units + num_groups)
  * combine records; num_partials partial-result slots live in the workspace; num_half_units of the units
  * have rows in one query tile only. num_half_units only picks a kernel variant (> 0: each such unit's KV
- * tiles alternate between both softmax warpgroups, which merge their two partial results at the end);
- * results are correct for any value, but the two variants round differently. */
+ * tiles alternate between both softmax warpgroups, which merge their two partial results at the end;
+ * == num_units: the unused second query buffer also serves as one more K/V slot); results are correct
+ * for any value below num_units, but the variants round differently. combine_row_blocks sizes the
+ * combine launch: the most thread blocks one combine record needs (one per row for a record of more than
+ * 16 chunks, else one per 8 rows), 0 for "unknown" (256 per record). A value below what the plan needs
+ * leaves rows unmerged and sets SEGPAGED_STATUS_UNIT. */
 typedef struct {
   int64_t num_units;
   int64_t num_groups;
   int64_t num_partials;
   int64_t num_half_units;
+  int64_t combine_row_blocks;
 } segpaged_plan_info;
 
 /* Text for an error code (static storage). */

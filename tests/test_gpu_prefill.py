@@ -73,6 +73,8 @@ SPLIT = {
                                                   seed=32), 1000),
     "mha-d64-p128-forced": (SMALL["mha-d64-p128"], 1000),
     "g2-p64-forced": (SMALL["g2-p64"], 1000),
+    # a decode-like batch: every unit a half unit (the variant with the second query buffer as a K/V slot)
+    "llama-decode8x16": (lambda: synth.llama_70b_decode(8, 16), None),
 }
 
 
@@ -95,6 +97,20 @@ def test_split_prefill_matches_oracle_every_row(name):
     r = _run(w, split_ctas=split)
     assert r.state[0].info["num_groups"] > 0, "expected a split plan"
     _every_row(name, w, r)
+
+
+def test_combine_grid_too_small_sets_status():
+    """A plan info whose combine_row_blocks is below what the plan needs leaves rows unmerged; the
+    combine launch reports it in the status word (SEGPAGED_STATUS_UNIT) instead of failing silently."""
+    w = SPLIT["split-short-q"][0]()
+    r = _run(w)
+    info = r.state[0].info
+    assert info["combine_row_blocks"] > 1
+    info["combine_row_blocks"] = 1
+    r.prefill(0)
+    torch.cuda.synchronize()
+    assert int(r.status.item()) & 8
+    r.status.zero_()
 
 
 def test_split_prefill_is_bit_identical_under_page_permutation():
