@@ -53,6 +53,8 @@ CASES = {name: SMALL[name] for name in ("tiny", "varlen-p16-g4", "mha-d64-p128",
 CASES["q0-mid-page"] = lambda: synth.custom("q0-mid-page", [(1000, 333), (77, 77), (600, 1)], 8, 2, 128, 64,
                                             [[(1, 0, 0), (0, 16, 100)], [(0, 3, 5), (1, 0, 0)], [(0, 700, 9), (0, 0, 600)]],
                                             seed=71)
+# a decode-like batch: every unit a half unit, split chunks with odd tile counts
+CASES["llama-decode8x16"] = lambda: synth.llama_70b_decode(8, 16)
 
 
 @pytest.mark.parametrize("name", list(CASES))

@@ -50,6 +50,7 @@ def _run(w, **kw):
 CASES = dict(SMALL)
 CASES["split-short-q"] = SPLIT["split-short-q"][0]
 CASES["qwen3-32b-lq64"] = lambda: synth.get("qwen3-32b-lq64")
+CASES["llama-decode8x16"] = SPLIT["llama-decode8x16"][0]
 
 
 @pytest.mark.parametrize("name", list(CASES))

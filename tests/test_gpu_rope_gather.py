@@ -109,6 +109,27 @@ def test_fragments_with_split_plan_match_oracle():
             "rope-split")
 
 
+def test_fragments_on_a_decode_batch_match_oracle():
+    """A decode-like batch (every unit a half unit, split chunks with odd tile counts) with several fragments
+    per sequence."""
+    w = synth.llama_70b_decode(8, 16)
+    rng = np.random.default_rng(64)
+    fo, fs, fc = _fragments(w, rng, per_seq=6)
+    r = _run(w, frags=(fo, fs, fc))
+    st = r.state[0]
+    assert st.info["num_groups"] > 0 and st.info["num_half_units"] == st.info["num_units"]
+    k, v = r.dense[0]
+    kn = orc.rope_fragment_keys(k.float().cpu().numpy(), w.cu_k(), fo, fs, fc)
+    pb = full_problem(w, 0, st.q.float().cpu().numpy(), kn, v.float().cpu().numpy())
+    items = np.array([(row, h) for row in range(w.total_q) for h in range(w.num_q_heads)], np.int64)
+    o_ref, lse_ref = lib().attention(pb, r.scale, items)
+    compare(st.o.float().cpu().numpy().reshape(-1, w.head_dim), st.lse.cpu().numpy().T.reshape(-1), o_ref, lse_ref,
+            "rope-decode-batch")
+    ref = lib().token_mass(pb, r.scale)
+    got = st.mass.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) <= MASS_RTOL * np.abs(ref) + MASS_ATOL)
+
+
 def test_fragment_prefill_is_bit_identical_under_page_permutation():
     w = SMALL["varlen-p16-g4"]()
     fr = _fragments(w, np.random.default_rng(63), per_seq=4)
