@@ -117,27 +117,6 @@ struct PrefillShared {
 // One pair of exponentials in every kExpCubicEvery runs on the FMA and integer pipes instead of MUFU (0: none).
 constexpr int kExpCubicEvery = 8;
 
-// 2^x for a pair on the FMA and integer pipes. Cody-Waite range reduction: n = floor(x) from a round-down add
-// of 1.5 * 2^23 (the sum's low mantissa bits hold n), f = x - n in [0, 1) (both steps exact), 2^f by a cubic
-// with minimal maximum relative error (fit_exp2_cubic.py beside this file: 7.5e-5), and n added to the exponent
-// bits. x is clamped to >= -126 first, so a masked logit (-inf) gives about 1.2e-38 instead of 0.
-__device__ __forceinline__ uint64_t exp2_cubic_pair(uint64_t x2) {
-  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t t = f2_add_rm(xc, f2_pack(kRound, kRound));
-  const uint64_t f = f2_sub(xc, f2_sub(t, f2_pack(kRound, kRound)));
-  uint64_t p = f2_fma(f2_pack(0x1.3f96a6p-4f, 0x1.3f96a6p-4f), f, f2_pack(0x1.cefc4ap-3f, 0x1.cefc4ap-3f));
-  p = f2_fma(p, f, f2_pack(0x1.64444cp-1f, 0x1.64444cp-1f));
-  p = f2_fma(p, f, f2_pack(0x1.fff632p-1f, 0x1.fff632p-1f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
-}
-
 // List position x of a unit -> page-table index.
 __device__ __forceinline__ int32_t unit_table_index(const int32_t* u, int32_t x) {
   return x < u[U_AN] ? x : u[U_B0] + (x - u[U_AN]);
