@@ -13,7 +13,8 @@
 //   warps 0-3   softmax for query tile 0, warps 4-7 softmax for query tile 1: one tile row per thread.
 //               tcgen05.ld of the S row, per-row bounds only on edge tiles, row max (3-input max),
 //               lazy O rescale (only when the running max grows by more than 2^8), exp2 on the MUFU
-//               unit, row sum and scaling in packed f32x2 arithmetic, P written back to TMEM as bf16 over
+//               unit (one pair in eight on the FMA pipe by a cubic, beside it), row sum and scaling in packed
+//               f32x2 arithmetic, P written back to TMEM as bf16 over
 //               S and published in two halves of 64 keys, and the epilogue (O / l -> bf16,
 //               LSE = ln 2 * (m + log2 l)).
 //   warp 8      producer (whole warp: page-table lookups; lane 0: barriers and TMA): claims units, TMA-loads both Q tiles (3-D map over [rows, Hq, D], box
