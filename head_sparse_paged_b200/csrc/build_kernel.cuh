@@ -63,19 +63,33 @@ __global__ void __launch_bounds__(256) build_scatter_kernel(BuildParams p) {
     const int64_t tok0 = (int64_t)lp * p.P;
     const int64_t src_base = (int64_t)p.cu_k[b];
     const uint4 zero = make_uint4(0, 0, 0, 0);
-    // V (and K without RoPE): plain copy.
-    for (int x = threadIdx.x; x < p.P * VPR; x += blockDim.x) {
-      const int row = x / VPR, vc = x % VPR;
-      const int64_t tok = tok0 + row;
-      const int64_t dst = ((int64_t)pid * p.P + row) * D + vc * 8;
-      uint4 vv = zero, kv = zero;
-      if (tok < L) {
-        const int64_t src = ((src_base + tok) * p.Hkv + kh) * D + vc * 8;
-        vv = *reinterpret_cast<const uint4*>(p.v_dense + src);
-        if (!ROPE) kv = *reinterpret_cast<const uint4*>(p.k_dense + src);
+    // V (and K without RoPE): plain copy. Each thread issues the loads of kUnroll vectors (read-only path)
+    // before their stores, so enough bytes are in flight per SM to cover the DRAM latency.
+    constexpr int kUnroll = 4;
+    const int nvec = p.P * VPR;
+    for (int x0 = threadIdx.x; x0 < nvec; x0 += blockDim.x * kUnroll) {
+      uint4 vv[kUnroll], kv[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int x = x0 + u * blockDim.x;
+        vv[u] = zero;
+        kv[u] = zero;
+        const int64_t tok = tok0 + x / VPR;
+        if (x < nvec && tok < L) {
+          const int64_t src = ((src_base + tok) * p.Hkv + kh) * D + (x % VPR) * 8;
+          vv[u] = __ldg(reinterpret_cast<const uint4*>(p.v_dense + src));
+          if (!ROPE) kv[u] = __ldg(reinterpret_cast<const uint4*>(p.k_dense + src));
+        }
       }
-      *reinterpret_cast<uint4*>(p.v_pool + dst) = vv;
-      if (!ROPE) *reinterpret_cast<uint4*>(p.k_pool + dst) = kv;
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int x = x0 + u * blockDim.x;
+        if (x < nvec) {
+          const int64_t dst = ((int64_t)pid * p.P + x / VPR) * D + (x % VPR) * 8;
+          *reinterpret_cast<uint4*>(p.v_pool + dst) = vv[u];
+          if (!ROPE) *reinterpret_cast<uint4*>(p.k_pool + dst) = kv[u];
+        }
+      }
     }
     if (ROPE) {
       constexpr int HPR = D / 16;  // vector pairs per row: (first-half chunk, second-half chunk)
