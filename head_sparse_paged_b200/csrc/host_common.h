@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -15,15 +16,17 @@ namespace host {
 
 constexpr int kMaxDevices = 64;
 
+// SM count of a device, looked up once per device (atomics: entry points may be called from several host
+// threads; a race only repeats the lookup).
 inline int device_sm_count(int dev) {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices];
   if (dev < 0 || dev >= kMaxDevices) return 0;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {

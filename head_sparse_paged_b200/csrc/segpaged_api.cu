@@ -400,14 +400,14 @@ template <int D, int P, int MODE, int HALF>
 int launch_prefill_v(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkn,
                      const CUtensorMap& tvn, const PrefillParams& p, int grid, cudaStream_t st) {
   using C = PrefillCfg<D, P, MODE == kModeRope>;
-  static bool configured[kMaxDevices] = {false};
+  static std::atomic<bool> configured[kMaxDevices];   // per device; a race only repeats the call
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
-  if (!configured[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
+  if (!configured[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(segpaged_prefill_kernel<D, P, MODE, HALF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return SEGPAGED_ERR_CUDA;
-    configured[dev] = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   segpaged_prefill_kernel<D, P, MODE, HALF><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, tv, tkn, tvn, p);
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;

@@ -96,14 +96,14 @@ namespace {
 template <int D, int P>
 int launch_mass(const CUtensorMap& tq, const CUtensorMap& tk, const MassParams& p, int grid, cudaStream_t st) {
   using C = MassCfg<D, P>;
-  static bool configured[kMaxDevices] = {false};
+  static std::atomic<bool> configured[kMaxDevices];   // per device; a race only repeats the call
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
-  if (!configured[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SEGPAGED_ERR_CUDA;
+  if (!configured[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(segpaged_mass_kernel<D, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return SEGPAGED_ERR_CUDA;
-    configured[dev] = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   segpaged_mass_kernel<D, P><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tk, p);
   return cudaGetLastError() == cudaSuccess ? SEGPAGED_OK : SEGPAGED_ERR_CUDA;

@@ -192,6 +192,10 @@ size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpage
  *   q (dev) [total_q, Hq, D] bf16.  k_pool, v_pool (dev) [num_pages, P, D] bf16.
  *   page_table (dev, int32) [page_table_len].
  *   plan (dev) [info->num_units + info->num_groups] records from segpaged_prefill_plan; info (host).
+ *     The plan must come from the same dims, lengths, classes and offsets as this call: its records
+ *     address query rows [0, total_q) with total_q = sum of q_len, and the kernel writes o and lse at
+ *     those rows without re-checking them against total_q (page-table entries are checked: see
+ *     SEGPAGED_STATUS_*). info must be the one the planner returned with it.
  *   softmax_scale: logits are scale * q.k (1/sqrt(D) in the usual case).
  *   o (dev) [total_q, Hq, D] bf16: O = softmax(logits over the visible keys) . V.
  *   lse (dev) [Hq, total_q] float: natural-log sum of exp(logits) over the visible keys.
