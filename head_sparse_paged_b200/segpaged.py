@@ -297,9 +297,9 @@ NOALLOC_MAX_UNITS = 16384
 def segpaged_attn_prefill_noalloc(dims: Dims, q, k_pool, v_pool, page_table, units_host, softmax_scale, o, lse,
                                   status=None, stream=None):
     """segpaged_attn_prefill for callers that cannot allocate device memory: the plan comes straight from
-    the host (int32 [n, 16] from segpaged_prefill_plan) and the library's own static device array holds
-    it and the work counter. At most NOALLOC_MAX_UNITS units, from a plan made with split_ctas = 0; calls
-    that overlap on the GPU race."""
+    the host (int32 [n, 32] records from segpaged_prefill_plan) and the library's own static device array
+    holds it and the work counter. At most NOALLOC_MAX_UNITS units, from a plan made with split_ctas = 0;
+    calls that overlap on the GPU race."""
     bf = torch.bfloat16
     units = np.ascontiguousarray(np.asarray(units_host, dtype=np.int32).reshape(-1, UNIT_FIELDS))
     r = _lib.segpaged_attn_prefill_noalloc(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]),
