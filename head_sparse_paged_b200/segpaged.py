@@ -136,6 +136,10 @@ def _dev(t: torch.Tensor | None, dtype=None, what=""):
         return None
     if not t.is_cuda:
         raise ValueError(f"{what}: expected a CUDA tensor")
+    # the library launches on, and encodes its tensor maps for, the current device
+    cur = torch.cuda.current_device()
+    if t.device.index is not None and t.device.index != cur:
+        raise ValueError(f"{what}: tensor on {t.device}, but the current device is cuda:{cur}")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{what}: expected {dtype}, got {t.dtype}")
     if not t.is_contiguous():

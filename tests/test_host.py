@@ -6,6 +6,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from head_sparse_paged_b200 import segpaged as sp
 from head_sparse_paged_b200 import synth
@@ -364,3 +365,25 @@ def test_append_plan_reads_old_keys_from_pool_and_new_keys_fresh(case, split):
                             if j >= q0)
             assert new[0] == first_vis // P
     assert np.all(seen == 1)
+
+
+def test_binding_rejects_tensors_off_the_current_device(monkeypatch):
+    """The library launches on the current device, so the binding refuses a tensor on another one before
+    any call (checked with a stand-in tensor: this machine has no GPU)."""
+    class FakeCudaTensor:
+        is_cuda = True
+        dtype = torch.bfloat16
+
+        def __init__(self, index):
+            self.device = torch.device("cuda", index)
+
+        def is_contiguous(self):
+            return True
+
+        def data_ptr(self):
+            return 4096
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="current device is cuda:0"):
+        sp._dev(FakeCudaTensor(1), torch.bfloat16, "q")
+    assert sp._dev(FakeCudaTensor(0), torch.bfloat16, "q").value == 4096
