@@ -406,3 +406,18 @@ def test_visible_flops_match_hand_count_and_enumeration():
             g, S, W = (int(x) for x in w.classes[0, b, kh])
             want += sum(len(orc.visible_keys(bool(g), S, W, i)) for i in range(L - Lq, L))
     assert visible_flops(w) == 4 * 64 * w.group * want
+
+
+def test_mass_pair_count_matches_enumeration():
+    """The token-mass leg's work count (one exponential per visible (query row, query head, key of the query
+    range)) against the oracle's explicit visible sets."""
+    import bench
+    w = synth.custom("ragged", [(1000, 300), (37, 37), (5, 0), (129, 1), (300, 300)], 8, 2, 64, 16,
+                     [[(0, 0, 100), (1, 0, 0)], [(0, 50, 3), (0, 2, 1)], [(1, 0, 0), (0, 1, 1)],
+                      [(0, 128, 1), (1, 0, 0)], [(0, 1000, 2), (0, 127, 129)]], seed=7)
+    want = 0
+    for b, (L, Lq) in enumerate(zip(w.ctx_lens, w.q_lens)):
+        for kh in range(w.num_kv_heads):
+            g, S, W = (int(x) for x in w.classes[0, b, kh])
+            want += sum(int((orc.visible_keys(bool(g), S, W, i) >= L - Lq).sum()) for i in range(L - Lq, L))
+    assert bench.mass_pairs(w, 0) == w.group * want
