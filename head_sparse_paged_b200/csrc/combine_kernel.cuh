@@ -38,6 +38,7 @@ struct CombineParams {
   __nv_bfloat16* o;        // [total_q, Hq, D]
   float* lse;              // [Hq, total_q]
   int32_t total_q, num_q_heads, log2_group;
+  int32_t num_partials;    // partial slots in part_o / part_lse
   int32_t row_blocks;      // gridDim.y: the most row blocks a record needs
   int32_t* status;         // nullable
 };
@@ -111,6 +112,13 @@ __global__ void __launch_bounds__(256) segpaged_combine_kernel(const CombinePara
     if (blockIdx.y == gridDim.y - 1 && threadIdx.x == 0 && p.status &&
         combine_blocks_of(npos, nsplit, G) > (int64_t)gridDim.y)
       atomicOr(p.status, kCombineStatusUnit);
+    // a record whose slots, rows or heads fall outside the call's arrays (not from this call's plan) is
+    // skipped and reported
+    if (part0 < 0 || nsplit < 0 || (int64_t)part0 + nsplit > p.num_partials || qrow0 < 0 ||
+        (int64_t)qrow0 + npos > p.total_q || (int64_t)(kvh + 1) * G > p.num_q_heads) {
+      if (blockIdx.y == 0 && threadIdx.x == 0 && p.status) atomicOr(p.status, kCombineStatusUnit);
+      continue;
+    }
     const int r = wide ? (int)blockIdx.y : (int)blockIdx.y * NW + warp;
     if ((wide ? r : (int)blockIdx.y * NW) >= rows) continue;     // uniform for the whole block
     const int tile = r >> 7, rr = r & 127;

@@ -85,6 +85,8 @@ struct PrefillParams {
   float* part_o;         // [partial slots][256 rows][D] fp32: O / l of one chunk of a split unit
   float* part_lse;       // [partial slots][256 rows] fp32: LSE of that chunk (natural log)
   int32_t total_q, num_q_heads, num_pages, log2_group;
+  int32_t num_partials;  // partial slots in part_o / part_lse
+  int32_t num_seqs;      // sequences of the call (RoPE: entries of frags.offs minus one)
   float scale_log2;      // softmax_scale * log2(e)
   RopeFragments frags;   // used by the ROPE variant only
   // fused append-and-attend: the new keys/values [total_q, Hkv, D] are read for the new-page tiles and
@@ -283,7 +285,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
               if (x < npages) {
                 const int32_t idx = unit_table_index(U, x);
                 my_pid = 0;
-                if (idx < 0 || idx >= U[U_TOTAL] || toff + idx >= p.page_table_len) {
+                if (idx < 0 || idx >= U[U_TOTAL] || toff + idx < 0 || toff + idx >= p.page_table_len) {
                   if (status) atomicOr(status, kStatusUnit);
                 } else {
                   my_pid = p.page_table[toff + idx];
@@ -507,7 +509,8 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
             const int32_t i = rest / VPR, vc = rest % VPR;
             const int32_t pos = pos0 + i, lp = pos / P;
             const int32_t idx = is_global ? lp : (lp < nsink ? lp : nsink + (lp - w0));
-            if (idx < 0 || idx >= total || toff + idx >= p.page_table_len || qrow + i >= p.total_q) {
+            if (idx < 0 || idx >= total || toff + idx < 0 || toff + idx >= p.page_table_len || qrow + i < 0 ||
+                qrow + i >= p.total_q || kvh < 0 || kvh >= p.num_kv_heads) {
               if (status) atomicOr(status, kStatusUnit);
               continue;
             }
@@ -552,7 +555,10 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         }
         const int32_t t0 = u[U_T0], an = u[U_AN], b0 = u[U_B0], nsink = u[U_NSINK], w0 = u[U_W0];
         const int32_t npages = u[U_AN] + u[U_BN];
-        const int32_t flo = p.frags.offs[u[U_SEQ]], fhi = p.frags.offs[u[U_SEQ] + 1];
+        // a sequence index outside the call (a record from another plan) rotates nothing and is reported
+        const bool seq_ok = u[U_SEQ] >= 0 && u[U_SEQ] < p.num_seqs;
+        if (!seq_ok && status && tid == 0) atomicOr(status, kStatusUnit);
+        const int32_t flo = seq_ok ? p.frags.offs[u[U_SEQ]] : 0, fhi = seq_ok ? p.frags.offs[u[U_SEQ] + 1] : 0;
         const int32_t nfr = fhi - flo;
         const bool in_smem = nfr <= kRopeSmemFragments;
         rope_bar();                                // the previous unit's searches are done
@@ -866,6 +872,12 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         if (two_o) ++mlcnt;
       };
       const int32_t part = u[U_PART];
+      if (part >= p.num_partials) {
+        // a record that names a partial slot the workspace does not have (not from this call's plan)
+        if (status && quarter == 0 && lane == 0) atomicOr(status, kStatusUnit);
+        release();
+        continue;
+      }
       if (part >= 0) {
         // one chunk of a split unit: O / l in fp32 and the chunk's LSE, for the combine pass; a row that
         // saw no visible key in this chunk writes O = 0 and LSE = -inf
@@ -889,6 +901,10 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       }
       const float inv_l = 1.0f / l_run;
       const int64_t qrow = (int64_t)u[U_QROW] + pslot;
+      // a row or head outside the call's outputs (a record from another plan) is skipped and reported
+      const bool in_range = qrow >= 0 && qrow < p.total_q && head >= 0 && head < p.num_q_heads;
+      if (valid_row && !in_range && status) atomicOr(status, kStatusUnit);
+      const bool store_row = valid_row && in_range;
       __nv_bfloat16* orow = p.o + (qrow * p.num_q_heads + head) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -898,13 +914,13 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
 #pragma unroll
         for (int k = 0; k < 16; ++k)
           w[k] = ptx::pack_bf16x2(__uint_as_float(r[2 * k]) * inv_l, __uint_as_float(r[2 * k + 1]) * inv_l);
-        if (valid_row) {
+        if (store_row) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
-      if (valid_row) p.lse[(int64_t)head * p.total_q + qrow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (store_row) p.lse[(int64_t)head * p.total_q + qrow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       release();
     }
   }

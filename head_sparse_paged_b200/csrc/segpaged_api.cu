@@ -311,6 +311,12 @@ int64_t plan_units(const segpaged_dims* dims, const int32_t* ctx_len, const int3
   std::stable_sort(out.begin(), out.end(),
                    [&](const segpaged_unit& a, const segpaged_unit& b) { return bucket(a) > bucket(b); });
   if (info) {
+    info->total_q = qrow;
+    info->page_table_len = B > 0 ? page_table_offs[B * H] : 0;
+    info->num_q_heads = dims->num_q_heads;
+    info->num_kv_heads = H;
+    info->head_dim = dims->head_dim;
+    info->page_size = P;
     info->num_units = (int64_t)out.size();
     info->num_groups = (int64_t)groups.size();
     info->num_partials = slots;
@@ -462,6 +468,11 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
     return SEGPAGED_ERR_DIMS;
   if (num_units == 0) return SEGPAGED_OK;
   if (!q || !k_pool || !v_pool || !page_table || !plan || !o || !lse || !workspace) return SEGPAGED_ERR_NULL;
+  // the plan must have been made for this call's shape: its records address rows, heads and table entries
+  if (info->total_q != total_q || info->num_q_heads != dims->num_q_heads || info->num_kv_heads != dims->num_kv_heads ||
+      info->head_dim != dims->head_dim || info->page_size != dims->page_size || page_table_len < info->page_table_len ||
+      info->num_half_units < 0 || info->num_half_units > num_units || (info->num_groups > 0) != (info->num_partials > 0))
+    return SEGPAGED_ERR_DIMS;
   if (workspace_bytes < segpaged_prefill_workspace_bytes(dims, info)) return SEGPAGED_ERR_CAPACITY;
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o) || !aligned16(plan) ||
       !aligned16(workspace))
@@ -505,6 +516,8 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   p.part_lse = reinterpret_cast<float*>(ws + kCounterBytes + partial_o_bytes(info->num_partials, D));
   p.total_q = total_q;
   p.num_q_heads = Hq;
+  p.num_partials = (int32_t)std::min<int64_t>(info->num_partials, INT32_MAX);
+  p.num_seqs = dims->num_seqs;
   p.num_pages = dims->num_pages;
   p.log2_group = log2_int(G);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
@@ -543,6 +556,7 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   c.lse = lse;
   c.total_q = total_q;
   c.num_q_heads = Hq;
+  c.num_partials = p.num_partials;
   c.log2_group = p.log2_group;
   c.status = status;
   const int64_t rb = info->combine_row_blocks;
@@ -636,6 +650,17 @@ extern "C" int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const vo
   // The static array holds no partial results, so split plans (chunks or combine records) are refused.
   for (int64_t i = 0; i < num_units; ++i)
     if (units_host[i].v[U_PART] >= 0 || units_host[i].v[U_NSPLIT] > 0) return SEGPAGED_ERR_UNSUPPORTED;
+  // Every unit must stay inside this call's arrays: its rows in [0, total_q), its KV head in [0, Hkv), its
+  // page-table entries in [0, page_table_len), at most two query tiles of positions.
+  const int32_t npos_tile = 128 / (dims->num_q_heads / dims->num_kv_heads);
+  for (int64_t i = 0; i < num_units; ++i) {
+    const int32_t* u = units_host[i].v;
+    const int32_t cap = u[U_HALF] ? npos_tile : 2 * npos_tile;
+    if (u[U_QROW] < 0 || u[U_NPOS] < 0 || u[U_NPOS] > cap || (int64_t)u[U_QROW] + u[U_NPOS] > total_q ||
+        u[U_KVH] < 0 || u[U_KVH] >= dims->num_kv_heads || u[U_TOFF] < 0 || u[U_TOTAL] < 0 ||
+        (int64_t)u[U_TOFF] + u[U_TOTAL] > page_table_len || u[U_NTILES] < 0 || u[U_T0] != 0 || u[U_NNEW] != 0)
+      return SEGPAGED_ERR_DIMS;
+  }
   int32_t* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch))) return rc;
   int32_t* units_dev = scratch + kNoAllocUnitOffset;
@@ -651,6 +676,12 @@ extern "C" int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const vo
   info.num_half_units = 0;
   for (int64_t i = 0; i < num_units; ++i) info.num_half_units += units_host[i].v[U_HALF] ? 1 : 0;
   info.combine_row_blocks = 0;
+  info.total_q = total_q;
+  info.page_table_len = page_table_len;
+  info.num_q_heads = dims->num_q_heads;
+  info.num_kv_heads = dims->num_kv_heads;
+  info.head_dim = dims->head_dim;
+  info.page_size = dims->page_size;
   return segpaged_attn_prefill(dims, q, total_q, k_pool, v_pool, page_table, page_table_len,
                                reinterpret_cast<const segpaged_unit*>(units_dev), &info, softmax_scale, o, lse,
                                scratch, kNoAllocUnitOffset * sizeof(int32_t), status, stream);

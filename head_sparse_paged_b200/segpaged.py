@@ -39,7 +39,12 @@ class SegPagedError(RuntimeError):
 
 class _PlanInfo(ctypes.Structure):
     _fields_ = [("num_units", ctypes.c_int64), ("num_groups", ctypes.c_int64), ("num_partials", ctypes.c_int64),
-                ("num_half_units", ctypes.c_int64), ("combine_row_blocks", ctypes.c_int64)]
+                ("num_half_units", ctypes.c_int64), ("combine_row_blocks", ctypes.c_int64),
+                ("total_q", ctypes.c_int64), ("page_table_len", ctypes.c_int64), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32)]
+
+
+PLAN_INFO_FIELDS = tuple(name for name, _ in _PlanInfo._fields_)
 
 
 class _Dims(ctypes.Structure):
@@ -189,8 +194,8 @@ def segpaged_build(dims: Dims, k_dense, v_dense, cu_seqlens_k, q_len, cls, page_
 
 
 def _info(d: dict) -> _PlanInfo:
-    return _PlanInfo(int(d["num_units"]), int(d["num_groups"]), int(d["num_partials"]), int(d.get("num_half_units", 0)),
-                     int(d.get("combine_row_blocks", 0)))
+    """The C struct of a plan-info dict as segpaged_prefill_plan returns it (every field required)."""
+    return _PlanInfo(*(int(d[name]) for name in PLAN_INFO_FIELDS))
 
 
 def _plan(fn, name, dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas):
@@ -206,8 +211,7 @@ def _plan(fn, name, dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas
     n2 = fn(ctypes.byref(d), _hp(L), _hp(Lq), _hp(c), _hp(offs), int(split_ctas), _hp(units), n, ctypes.byref(info))
     if n2 < 0:
         raise SegPagedError(int(n2), name)
-    return units[:n], {"num_units": info.num_units, "num_groups": info.num_groups, "num_partials": info.num_partials,
-                       "num_half_units": info.num_half_units, "combine_row_blocks": info.combine_row_blocks}
+    return units[:n], {name: int(getattr(info, name)) for name in PLAN_INFO_FIELDS}
 
 
 def segpaged_prefill_plan(dims: Dims, ctx_len, q_len, cls, page_table_offs, split_ctas: int = 0):

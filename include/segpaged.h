@@ -98,13 +98,25 @@ typedef struct {
  * for any value below num_units, but the variants round differently. combine_row_blocks sizes the
  * combine launch: the most thread blocks one combine record needs (one per row for a record of more than
  * 16 chunks, else one per 8 rows), 0 for "unknown" (256 per record). A value below what the plan needs
- * leaves rows unmerged and sets SEGPAGED_STATUS_UNIT. */
+ * leaves rows unmerged and sets SEGPAGED_STATUS_UNIT.
+ * The last six fields record the call the plan was made for: its records address query rows
+ * [0, total_q), query heads [0, num_q_heads) and page-table entries [0, page_table_len) (the planner's
+ * page_table_offs[B*Hkv]). The prefill entry points return SEGPAGED_ERR_DIMS before any launch when the
+ * call's total_q, num_q_heads, num_kv_heads, head_dim or page_size differ from them or its page table is
+ * shorter, and the kernels skip (and report with SEGPAGED_STATUS_UNIT) any output row, head or partial
+ * slot a record names outside the call's arrays. */
 typedef struct {
   int64_t num_units;
   int64_t num_groups;
   int64_t num_partials;
   int64_t num_half_units;
   int64_t combine_row_blocks;
+  int64_t total_q;
+  int64_t page_table_len;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
 } segpaged_plan_info;
 
 /* Text for an error code (static storage). */
@@ -192,10 +204,11 @@ size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpage
  *   q (dev) [total_q, Hq, D] bf16.  k_pool, v_pool (dev) [num_pages, P, D] bf16.
  *   page_table (dev, int32) [page_table_len].
  *   plan (dev) [info->num_units + info->num_groups] records from segpaged_prefill_plan; info (host).
- *     The plan must come from the same dims, lengths, classes and offsets as this call: its records
- *     address query rows [0, total_q) with total_q = sum of q_len, and the kernel writes o and lse at
- *     those rows without re-checking them against total_q (page-table entries are checked: see
- *     SEGPAGED_STATUS_*). info must be the one the planner returned with it.
+ *     The plan must come from the same dims, lengths, classes and offsets as this call, and info must be
+ *     the one the planner returned with it. A call whose total_q, heads, head_dim, page_size or page
+ *     table length disagree with info returns SEGPAGED_ERR_DIMS before any launch; a record that still
+ *     names a row, head, page-table entry or partial slot outside the call's arrays (records from another
+ *     plan than info's) is skipped and sets SEGPAGED_STATUS_UNIT.
  *   softmax_scale: logits are scale * q.k (1/sqrt(D) in the usual case).
  *   o (dev) [total_q, Hq, D] bf16: O = softmax(logits over the visible keys) . V.
  *   lse (dev) [Hq, total_q] float: natural-log sum of exp(logits) over the visible keys.
@@ -281,7 +294,9 @@ int segpaged_attn_prefill_rope(const segpaged_dims* dims, const void* q, int32_t
  *   units_host (host) [num_units] straight from segpaged_prefill_plan called with split_ctas = 0 (a
  *     plan with split units returns SEGPAGED_ERR_UNSUPPORTED); it is copied on `stream` into a
  *     library-owned device array, so keep it unchanged until the stream has passed this call
- *     (a pageable buffer is staged before the call returns);
+ *     (a pageable buffer is staged before the call returns). Every unit is checked on the host first:
+ *     one whose query rows, KV head or page-table entries fall outside this call's total_q, dims or
+ *     page_table_len returns SEGPAGED_ERR_DIMS before anything is enqueued;
  *   no workspace arguments.
  * The library-owned array is a static device array of 2 MiB that every GPU loading the library keeps
  * until the process exits; it holds at most 16384 units (more return SEGPAGED_ERR_CAPACITY). The

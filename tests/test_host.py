@@ -198,6 +198,63 @@ def test_noalloc_refuses_split_plans():
     assert rc == -9
 
 
+def test_prefill_rejects_a_plan_made_for_another_call():
+    """A plan records the shape of the call it was made for (rows, heads, head_dim, page size, page-table
+    length); a call that disagrees gets SEGPAGED_ERR_DIMS before anything is enqueued, and the allocation-free
+    entry point checks every unit of its host plan the same way. Only calls the host checks refuse are made
+    here: the device addresses are fake (aligned, never dereferenced)."""
+    dims = sp.Dims(2, 8, 2, 64, 16, 4000)
+    ctx, ql = [900, 300], [200, 64]
+    cls = [[(1, 0, 0), (0, 4, 64)], [(0, 8, 100), (1, 0, 0)]]
+    _, _, per = sp.segpaged_pages_bytes(dims, ctx, ql, cls)
+    offs = np.concatenate([[0], np.cumsum(per)]).astype(np.int32)
+    units, info = sp.segpaged_prefill_plan(dims, ctx, ql, cls, offs, 0)
+    assert info["total_q"] == 264 and info["page_table_len"] == int(offs[-1])
+    assert (info["num_q_heads"], info["num_kv_heads"], info["head_dim"], info["page_size"]) == (8, 2, 64, 16)
+    lib = sp.library()
+    fake = ctypes.c_void_p(1 << 24)
+
+    def prefill(d, total_q, table_len, inf):
+        return lib.segpaged_attn_prefill(ctypes.byref(d.c()), fake, total_q, fake, fake, fake, table_len, fake,
+                                         ctypes.byref(sp._info(inf)), 0.125, fake, fake, fake, 1 << 26, None, None)
+
+    # the plan of a longer query range (264 rows) given to a call with fewer rows, or more
+    assert prefill(dims, 200, int(offs[-1]), info) == -2
+    assert prefill(dims, 300, int(offs[-1]), info) == -2
+    # a page table shorter than the entries the plan addresses
+    assert prefill(dims, 264, int(offs[-1]) - 1, info) == -2
+    # other head counts, head_dim or page size than the plan's
+    for other in (sp.Dims(2, 16, 2, 64, 16, 4000), sp.Dims(2, 8, 4, 64, 16, 4000), sp.Dims(2, 8, 2, 128, 16, 4000),
+                  sp.Dims(2, 8, 2, 64, 32, 4000)):
+        assert prefill(other, 264, int(offs[-1]), info) == -2
+    # an info that disagrees with itself: half units beyond the units, combine records without partial slots
+    assert prefill(dims, 264, int(offs[-1]), dict(info, num_half_units=info["num_units"] + 1)) == -2
+    assert prefill(dims, 264, int(offs[-1]), dict(info, num_groups=1, num_partials=0)) == -2
+    # the same rules through the other prefill entry points
+    assert lib.segpaged_attn_prefill_append(ctypes.byref(dims.c()), fake, 200, fake, fake, fake, fake, fake,
+                                            int(offs[-1]), fake, ctypes.byref(sp._info(info)), 0.125, fake, fake, fake,
+                                            1 << 26, None, None) == -2
+    assert lib.segpaged_attn_prefill_rope(ctypes.byref(dims.c()), fake, 200, fake, fake, fake, int(offs[-1]), fake,
+                                          ctypes.byref(sp._info(info)), 0.125, fake, fake, fake, fake, fake, fake,
+                                          1 << 26, None, None) == -2
+
+    # allocation-free entry point: every unit is checked against the call's rows, heads and table
+    def noalloc(recs, total_q, table_len, d=dims):
+        recs = np.ascontiguousarray(recs, dtype=np.int32)
+        return lib.segpaged_attn_prefill_noalloc(ctypes.byref(d.c()), fake, total_q, fake, fake, fake, table_len,
+                                                 recs.ctypes.data_as(ctypes.c_void_p), len(recs), 0.125, fake, fake,
+                                                 None, None)
+
+    U_QROW, U_KVH, U_TOFF = 0, 3, 4
+    assert noalloc(units, 200, int(offs[-1])) == -2                     # rows past the call's 200
+    assert noalloc(units, 264, int(offs[-1]) - 1) == -2                 # entries past the call's table
+    assert noalloc(units, 264, int(offs[-1]), sp.Dims(2, 8, 1, 64, 16, 4000)) == -2   # KV head 1 of 1
+    for field, value in ((U_QROW, -1), (U_KVH, 2), (U_KVH, -1), (U_TOFF, -3)):
+        bad = units.copy()
+        bad[len(bad) // 2, field] = value
+        assert noalloc(bad, 264, int(offs[-1])) == -2, (field, value)
+
+
 @pytest.mark.parametrize("name", ["tiny", "mistral-7b", "llama-3.3-70b", "qwen3-32b"])
 def test_plan_workloads(name):
     w = synth.get(name)
