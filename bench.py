@@ -6,10 +6,11 @@ work planning on the host, the build scatter of the layer's K/V into its pages, 
 paged prefill. The metric is visible-KV TFLOP/s: 4 * D * sum |V(i)| over every (query row, query head)
 of every layer, divided by the step time (CUDA events, max over ranks).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference|dense]
 
-Under torchrun every rank runs its own replica of the workload (rank-specific seeds, no data-path
-collective: weak scaling); rank 0 prints one JSON line.
+With N > 1 every rank runs its own replica of the workload on its own GPU (rank-specific seeds, no
+data-path collective: weak scaling); rank 0 prints one JSON line. Under torchrun the ranks come from its
+environment; run plainly with --gpus N, bench.py starts the N ranks itself.
 """
 from __future__ import annotations
 
@@ -57,8 +58,13 @@ def parse_args(argv=None):
                     help="tokens per reused fragment in the gather-time RoPE measurement")
     ap.add_argument("--topk-frac", type=float, default=0.25,
                     help="share of each sequence's query tokens the top-k selection keeps")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the one-layer Qwen3-32B- and Llama-3.3-70B-shaped prefill measurements")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip the dense-layout baseline (explicit mask) on an all-global and a mixed layer")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle sample")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the oracle sample (per step in --impl reference)")
     return ap.parse_args(argv)
 
 
@@ -107,23 +113,17 @@ def kernel_source_hash() -> str:
 
 
 def traffic_per_launch(workload: str):
-    """DRAM bytes per prefill launch from the committed ncu summary, if it was taken on the current
-    kernel sources for this workload; else None."""
-    p = os.path.join(ROOT, "profiles", f"prefill_traffic_{workload}.md")
+    """DRAM bytes per prefill launch of this workload from profiles/prefill_traffic_<workload>.json (an ncu
+    capture summary), if it was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"prefill_traffic_{workload}.json")
     if not os.path.exists(p):
         return None
-    vals = {}
     with open(p) as f:
-        for line in f:
-            if ":" in line and line.strip().startswith("- "):
-                k, v = line.strip()[2:].split(":", 1)
-                vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_sources_sha256") != kernel_source_hash():
+        d = json.load(f)
+    if d.get("kernel_sources_sha256") != kernel_source_hash():
         return None
-    try:
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    v = d.get("dram_bytes_per_launch")
+    return float(v) if v is not None else None
 
 
 class ClockSampler:
@@ -193,7 +193,7 @@ def oracle_sample(w, inputs_for_head, seconds: float, seed: int = 0):
     every layer class present, in rounds, until the time budget is spent. Returns (visible TFLOP/s,
     sample description, threads)."""
     import numpy as np
-    from head_sparse_paged_b200.runner import visible_counts
+    from head_sparse_paged_b200.counts import visible_counts
     from oracle import reference as orc
 
     lib = orc.OracleLib()
@@ -277,10 +277,10 @@ def run_reference(args, rank, world):
     """The oracle as it stands, timed on the host cores, on this workload's config and metric."""
     if rank != 0:
         return 0
-    from head_sparse_paged_b200.runner import visible_flops
+    from head_sparse_paged_b200.counts import visible_flops
     w = rank_workload(args.workload, 0)
     get = oracle_head_inputs_from_synth(w)
-    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.2, min(20.0, 150.0 / max(1, args.steps + args.warmup), args.cpu_seconds))
     for _ in range(args.warmup):
         oracle_sample(w, get, per_step / 4, seed=1)
     vals = []
@@ -291,11 +291,16 @@ def run_reference(args, rank, world):
     value = statistics.median(vals)
     flops = visible_flops(w)
     ms = flops / (value * 1e12) * 1e3
+    from oracle import reference as orc
+    stored = 0
+    for li in range(w.layers):
+        c = w.classes[li]
+        stored += orc.pages_bytes(w.cu_k(), w.cu_q(), c[..., 0], c[..., 1], c[..., 2], w.page_size, w.head_dim)[0]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
+        "config": workload_config(w, world, stored),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"each step: {desc}; step time extrapolated by visible FLOPs"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -304,69 +309,83 @@ def run_reference(args, rank, world):
     return 0
 
 
+def dense_chunk_rows(w, L: int) -> int:
+    """Query rows per SDPA call of the dense-layout baseline: each call's boolean mask stays near 2 GB."""
+    return max(1, int(2e9 // (w.num_q_heads * L)))
+
+
+def dense_layer_ms(w, li, q, k_all, v_all, device):
+    """Attention time of one layer in the dense layout: every head keeps its full context as a dense
+    [Hq, L, D] K/V and visibility is an explicit boolean mask given to PyTorch's scaled_dot_product_attention
+    (the masked slow path SegPagedAttention avoids). Query rows are chunked (dense_chunk_rows); each chunk's
+    mask is built before its call and only the attention calls are timed, each between its own CUDA events,
+    after one untimed pass."""
+    import torch
+    import torch.nn.functional as F
+    G, D = w.group, w.head_dim
+    scale = 1.0 / math.sqrt(D)
+    cq, ck = w.cu_q(), w.cu_k()
+    ms = 0.0
+    for b in range(w.num_seqs):
+        L, Lq = w.ctx_lens[b], w.q_lens[b]
+        if Lq == 0:
+            continue
+        kk = k_all[ck[b]:ck[b + 1]].transpose(0, 1).repeat_interleave(G, dim=0)[None]   # [1, Hq, L, D]
+        vv = v_all[ck[b]:ck[b + 1]].transpose(0, 1).repeat_interleave(G, dim=0)[None]
+        qq = q[cq[b]:cq[b + 1]].transpose(0, 1)[None]                                      # [1, Hq, Lq, D]
+        cls = torch.from_numpy(w.classes[li, b]).to(device).repeat_interleave(G, dim=0)  # [Hq, 3]
+        glob, S, W = cls[:, 0, None, None] != 0, cls[:, 1, None, None], cls[:, 2, None, None]
+        j = torch.arange(L, device=device)[None, None, :]
+        chunk = dense_chunk_rows(w, L)
+        pairs = []
+        for rep in range(2):          # the first pass warms up; only the second is timed
+            for r0 in range(0, Lq, chunk):
+                i = (L - Lq + torch.arange(r0, min(r0 + chunk, Lq), device=device))[None, :, None]
+                m = ((j <= i) & (glob | (j < S) | (j > i - W)))[None]
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                F.scaled_dot_product_attention(qq[:, :, r0:r0 + m.shape[2]], kk, vv, attn_mask=m, scale=scale)
+                e1.record()
+                if rep == 1:
+                    pairs.append((e0, e1))
+                del m
+        torch.cuda.synchronize()
+        ms += sum(a.elapsed_time(b_) for a, b_ in pairs)
+        del kk, vv
+    return ms
+
+
 def run_dense(args, rank, world, local):
-    """Dense-layout baseline on the same GPU: every head keeps its full context as a dense [Hq, L, D] K/V and
-    the sink-plus-window visibility is an explicit boolean mask given to PyTorch's scaled_dot_product_attention
-    (the masked slow path SegPagedAttention avoids). One layer of each kind is timed with CUDA events: query
-    rows are chunked so each mask stays near 2 GB, each chunk's mask is built before its call, and only the
-    attention calls are timed, each between its own events. Per-layer times are weighted by how many layers
-    of that kind the workload has."""
+    """Dense-layout baseline on the same GPU (dense_layer_ms), one layer of each kind (number of global heads),
+    weighted by how many layers of that kind the workload has."""
     if rank != 0:
         return 0
     import torch
-    import torch.nn.functional as F
     from head_sparse_paged_b200 import synth
-    from head_sparse_paged_b200.runner import visible_flops
+    from head_sparse_paged_b200.counts import visible_flops
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = rank_workload(args.workload, 0)
     kinds = {}
     for li in range(w.layers):
         kinds.setdefault(int(w.classes[li][..., 0].sum()), []).append(li)
-    G, D = w.group, w.head_dim
-    scale = 1.0 / math.sqrt(D)
     per_layer_ms, ms_step = {}, 0.0
     _, k_all, v_all = synth.layer_inputs(w, 0, device=device)
-    cq, ck = w.cu_q(), w.cu_k()
     for key, lis in kinds.items():
         li = lis[0]
         q = synth.layer_inputs(w, li, device=device, parts="q")[0]
         if w.layers == 1:
             _, k_all, v_all = synth.layer_inputs(w, li, device=device)
-        ms_layer = 0.0
-        for b in range(w.num_seqs):
-            L, Lq = w.ctx_lens[b], w.q_lens[b]
-            if Lq == 0:
-                continue
-            kk = k_all[ck[b]:ck[b + 1]].transpose(0, 1).repeat_interleave(G, dim=0)[None]   # [1, Hq, L, D]
-            vv = v_all[ck[b]:ck[b + 1]].transpose(0, 1).repeat_interleave(G, dim=0)[None]
-            qq = q[cq[b]:cq[b + 1]].transpose(0, 1)[None]                                      # [1, Hq, Lq, D]
-            cls = torch.from_numpy(w.classes[li, b]).to(device).repeat_interleave(G, dim=0)  # [Hq, 3]
-            glob, S, W = cls[:, 0, None, None] != 0, cls[:, 1, None, None], cls[:, 2, None, None]
-            j = torch.arange(L, device=device)[None, None, :]
-            chunk = max(1, int(2e9 // (w.num_q_heads * L)))
-            pairs = []
-            for rep in range(2):          # the first pass warms up; only the second is timed
-                for r0 in range(0, Lq, chunk):
-                    i = (L - Lq + torch.arange(r0, min(r0 + chunk, Lq), device=device))[None, :, None]
-                    m = ((j <= i) & (glob | (j < S) | (j > i - W)))[None]
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record()
-                    F.scaled_dot_product_attention(qq[:, :, r0:r0 + m.shape[2]], kk, vv, attn_mask=m, scale=scale)
-                    e1.record()
-                    if rep == 1:
-                        pairs.append((e0, e1))
-                    del m
-            torch.cuda.synchronize()
-            ms_layer += sum(a.elapsed_time(b_) for a, b_ in pairs)
-            del kk, vv
+        ms_layer = dense_layer_ms(w, li, q, k_all, v_all, device)
         per_layer_ms[f"{len(lis)} layers with {key} global heads"] = ms_layer
         ms_step += ms_layer * len(lis)
     flops = visible_flops(w)
     line = {
         "impl": "dense", "metric": METRIC, "value": flops / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
         "n_gpus": 1, "ms_per_step": ms_step, "ms_per_layer": ms_step / w.layers, "higher_is_better": True,
-        "dtype": "bf16", "data": "synthetic", "config": workload_config(w), "dense_ms_by_layer_kind": per_layer_ms,
+        "dtype": "bf16", "data": "synthetic", "dense_ms_by_layer_kind": per_layer_ms,
+        "query_chunk_rows": {str(L): dense_chunk_rows(w, L) for L in sorted(set(w.ctx_lens))},
+        "workload": w.name,
         "note": "PyTorch SDPA with an explicit boolean mask over dense K/V of every head at full context; "
                 "value = visible FLOPs / time, so it is directly comparable with the SegPaged line",
     }
@@ -374,16 +393,23 @@ def run_dense(args, rank, world, local):
     return 0
 
 
-def workload_config(w):
+def workload_config(w, world: int, stored_bytes: int):
+    """The `config` object of every arm's line: the workload, how it is replicated, and why L2 cannot hold it.
+    stored_bytes: K+V page bytes of all layers (the page pool, which each step streams)."""
     return {"workload": w.name, "description": w.description, "layers": w.layers, "seq_lens": list(w.ctx_lens),
             "q_lens": list(w.q_lens), "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
-            "head_dim": w.head_dim, "page_size": w.page_size, "page_order": w.page_order}
+            "head_dim": w.head_dim, "page_size": w.page_size, "page_order": w.page_order,
+            "global_batch": w.num_seqs * world, "parallelism": f"replicas x{world}" if world > 1 else "single",
+            "l2": f"inputs larger than L2 (page pool {stored_bytes / 1e9:.2f} GB per replica, all read every step)"
+                  if stored_bytes > 126e6 else f"page pool {stored_bytes / 1e6:.1f} MB fits in L2",
+            "dense_kv_source": "shared by all layers" if w.layers > 1 else "per layer"}
 
 
 def run_ours(args, rank, world, local):
     import numpy as np
     import torch
-    from head_sparse_paged_b200.runner import Runner, visible_flops
+    from head_sparse_paged_b200.counts import visible_flops
+    from head_sparse_paged_b200.runner import Runner
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -470,6 +496,14 @@ def run_ours(args, rank, world, local):
     if not args.no_append and runner.rope is None:
         append = measure_append(runner, args, device, flops_layer, prefill_total_ms / args.steps)
 
+    # the 32K-128K single-layer configurations and the dense-layout baseline, beside the headline (one GPU only)
+    workloads = None
+    if world == 1 and not args.no_workloads:
+        workloads = measure_workloads(args, device, [n for n in ("qwen3-32b", "llama-3.3-70b") if n != w.name])
+    dense_baseline = None
+    if world == 1 and not args.no_dense:
+        dense_baseline = measure_dense_baseline(runner, device, prefill_ms)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         def inputs(li, b, kh):
@@ -480,11 +514,8 @@ def run_ours(args, rank, world, local):
 
     if rank != 0:
         return 0
-    cfg = workload_config(w)
-    cfg.update({"global_batch": w.num_seqs * world, "parallelism": f"replicas x{world}" if world > 1 else "single",
-                "l2": f"inputs larger than L2 (page pool {runner.num_pages * w.page_size * w.head_dim * 4 / 1e9:.1f} GB, "
-                      f"stored per step {stored / 1e9:.2f} GB)",
-                "dense_kv_source": "shared by all layers" if runner.shared_dense else "per layer"})
+    cfg = workload_config(w, world, stored)
+    launches_layer = {li: 2 + (1 if runner.state[li].info["num_groups"] > 0 else 0) for li in runner.layers}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -500,32 +531,99 @@ def run_ours(args, rank, world, local):
                      "peak_source": f"{src} {peak_name}", "kernel": "segpaged_prefill_kernel"},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "workloads": workloads,
+        "dense_baseline": dense_baseline,
         "token_mass": mass,
         "rope_gather": rope_gather,
         "append": append,
-        "gpu_launches": args.steps * n_layers * 2,
+        "gpu_launches": args.steps * sum(launches_layer.values()),
+        "gpu_launches_note": "per layer and step: build scatter, prefill, and the combine where the plan splits units",
         "clocks": clocks,
     }
     print(json.dumps(line))
     return 0
 
 
+def _roofline(w, flops: float, nbytes: float, ms: float, peaks: dict, tf_name: str, src: str):
+    """Bound (the slower of visible FLOPs at the tensor peak and algorithmic bytes at HBM bandwidth), achieved rate
+    and fraction of one launch that took `ms`."""
+    peak_tf, peak_bw = float(peaks[tf_name]), float(peaks["hbm_gbs"])
+    if nbytes / (peak_bw * 1e9) > flops / (peak_tf * 1e12):
+        ach = nbytes / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": peak_bw, "unit": "GB/s", "frac": ach / peak_bw,
+                "peak_source": f"{src} hbm_gbs"}
+    ach = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
+            "peak_source": f"{src} {tf_name}"}
+
+
+def measure_workloads(args, device, names):
+    """Prefill of one layer of each named workload (Qwen3-32B-shaped 128K and Llama-3.3-70B-shaped 16-32K batch),
+    set up through the same C ABI and timed like the headline's kernel: CUDA events around each launch (the
+    prefill, and the combine where the plan splits units), W warm-up launches, then K timed ones. These runs are
+    short bursts at full clock, so their fraction is taken against the burst GEMM peak."""
+    import torch
+    from head_sparse_paged_b200 import synth
+    from head_sparse_paged_b200.counts import visible_flops
+    from head_sparse_paged_b200.runner import Runner
+    peaks, src = load_peaks()
+    out = {}
+    for name in names:
+        w = synth.get(name)
+        r = Runner(w, device=device)
+        torch.cuda.synchronize()
+        r.check_status()
+        stream = torch.cuda.current_stream()
+        for _ in range(args.warmup):
+            r.prefill(0)
+        torch.cuda.synchronize()
+        ev = []
+        with ClockSampler(device.index if device.index is not None else 0) as clk:
+            for _ in range(args.steps):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                r.prefill(0)
+                b.record(stream)
+                ev.append((a, b))
+            torch.cuda.synchronize()
+        r.check_status()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+        flops = visible_flops(w, [0])
+        nbytes = r.state[0].stored_bytes + w.total_q * w.num_q_heads * (w.head_dim * 2 * 2 + 4)
+        rl = _roofline(w, flops, nbytes, ms, peaks, "bf16_tflops", src)
+        out[name] = {"prefill_ms": ms, "visible_tflop": flops / 1e12, "tflops": flops / (ms * 1e-3) / 1e12,
+                     "algorithmic_bytes": nbytes, **rl, "split_plan": r.state[0].info["num_groups"] > 0,
+                     "sm_mhz": clk.summary()["sm_mhz"], "launches": args.steps}
+        del r
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_dense_baseline(runner, device, prefill_ms):
+    """The dense-layout baseline (dense_layer_ms) on the first layer of each kind of the workload (all-global, mixed),
+    against the SegPaged prefill of the same layer from the timed steps."""
+    w = runner.w
+    out = {}
+    done = set()
+    for li in runner.layers:
+        kind = "all-global" if runner.state[li].cls[..., 0].all() else "mixed"
+        if kind in done:
+            continue
+        done.add(kind)
+        k, v = runner.dense_of(li)
+        ms = dense_layer_ms(w, li, runner.state[li].q, k, v, device)
+        ours = statistics.mean(prefill_ms[li])
+        out[kind] = {"layer": li, "dense_ms": ms, "segpaged_prefill_ms": ours, "ratio": ms / ours}
+    out["query_chunk_rows"] = {str(L): dense_chunk_rows(w, L) for L in sorted(set(w.ctx_lens))}
+    out["method"] = ("PyTorch scaled_dot_product_attention over dense K/V of every head at full context with an "
+                     "explicit boolean mask, query rows chunked so each mask stays near 2 GB, only the attention "
+                     "calls timed (CUDA events), after one untimed pass")
+    return out
+
+
 # MUFU peak for the token-mass pass: 16 ex2 per clock per SM (sm_100), 148 SMs, at the maximum SM clock.
 MUFU_EX2_PER_CLK_SM = 16
-
-
-def mass_pairs(w, layer):
-    """Visible (query row, query head, key of the query range) triples of one layer: one exp2 each."""
-    import numpy as np
-    total = 0
-    for b in range(w.num_seqs):
-        L, Lq = w.ctx_lens[b], w.q_lens[b]
-        j = np.arange(L - Lq, L, dtype=np.int64)
-        for kh in range(w.num_kv_heads):
-            g, S, W = (int(x) for x in w.classes[layer, b, kh])
-            n = (L - j) if g else np.where(j < S, L - j, np.minimum(L - j, W))
-            total += w.group * int(n.sum())
-    return total
 
 
 def measure_mass(runner, args, world, device):
@@ -538,6 +636,7 @@ def measure_mass(runner, args, world, device):
     k_per_seq = torch.tensor([max(1, int(round(args.topk_frac * l))) for l in w.q_lens], dtype=torch.int32,
                              device=device)
     selected = torch.empty(int(k_per_seq.sum().item()), dtype=torch.int32, device=device)
+    from head_sparse_paged_b200.counts import mass_pairs
     pairs = {li: mass_pairs(w, li) for li in runner.layers}
     for _ in range(args.warmup):
         for li in runner.layers:
@@ -780,9 +879,50 @@ def measure_e2e(runner, args, world, device, flops_step):
                       "layer by layer"}
 
 
+def _free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def _rank_entry(target, argv, env):
+    os.environ.update(env)
+    sys.exit(int(target(argv) or 0))
+
+
+def spawn_ranks(nprocs: int, target, argv) -> int:
+    """Runs target(argv) as ranks 0 .. nprocs-1 of one job on this node, each in a fresh process (spawn, so no
+    CUDA state is inherited) with the environment torchrun would give it (RANK, LOCAL_RANK, WORLD_SIZE,
+    MASTER_ADDR=127.0.0.1, a free MASTER_PORT). Rank r uses GPU r. Returns the largest exit code of the ranks."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = []
+    for r in range(nprocs):
+        env = {"RANK": str(r), "LOCAL_RANK": str(r), "WORLD_SIZE": str(nprocs), "LOCAL_WORLD_SIZE": str(nprocs),
+               "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)}
+        p = ctx.Process(target=_rank_entry, args=(target, list(argv), env))
+        p.start()
+        procs.append(p)
+    rc = 0
+    for p in procs:
+        p.join()
+        code = p.exitcode if p.exitcode is not None else 1
+        rc = max(rc, code if code >= 0 else 1)
+    return rc
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     args = parse_args(argv)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # started plainly with --gpus N: run the N ranks here, one process and one GPU each
+        return spawn_ranks(args.gpus, main, argv)
     rank, world, local = dist_env()
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but the job has {world} ranks", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args, rank, world)
     if args.impl == "dense":
@@ -792,6 +932,7 @@ def main(argv=None):
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local)
+        # NCCL carries only the reporting barrier and max-over-ranks reduction: the replicas share no data
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
         return run_ours(args, rank, world, local)

@@ -16,6 +16,7 @@ import torch
 
 from . import segpaged as sp
 from . import synth
+from .counts import visible_counts, visible_flops  # noqa: F401  (re-exported)
 
 
 @dataclass
@@ -261,25 +262,3 @@ class Runner:
         s = int(self.status.item())
         if s:
             raise RuntimeError(f"device status word {s:#x}")
-
-
-def visible_counts(w: synth.Workload, layer: int, b: int, kh: int) -> np.ndarray:
-    """|V(i)| for every query position of (sequence b, KV head kh) of a layer."""
-    L, Lq = w.ctx_lens[b], w.q_lens[b]
-    i = np.arange(L - Lq, L, dtype=np.int64)
-    g, S, W = (int(x) for x in w.classes[layer, b, kh])
-    if g:
-        return i + 1
-    sink = np.minimum(S, i + 1)
-    lo = np.maximum(i - W + 1, 0)
-    return sink + (i + 1 - lo) - np.clip(sink - lo, 0, None)
-
-
-def visible_flops(w: synth.Workload, layers=None) -> float:
-    """4 * D * sum over (sequence, query head, query row) of |V(i)|: the algorithmic FLOPs of prefill."""
-    total = 0.0
-    for li in (range(w.layers) if layers is None else layers):
-        for b in range(w.num_seqs):
-            for kh in range(w.num_kv_heads):
-                total += 4.0 * w.head_dim * w.group * float(visible_counts(w, li, b, kh).sum())
-    return total

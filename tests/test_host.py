@@ -450,7 +450,7 @@ def test_visible_flops_match_hand_count_and_enumeration():
     """The reported metric's numerator, 4 * D * sum |V(i)| over (query row, query head), against the tiny
     layer counted by hand (global rows 192..255 see i + 1 keys; local rows see 4 sink + 64 window keys, which
     do not meet) and against the oracle's explicit visible sets on ragged shapes."""
-    from head_sparse_paged_b200.runner import visible_flops
+    from head_sparse_paged_b200.counts import visible_flops
     w = synth.tiny()
     assert visible_flops(w) == 4 * 64 * 2 * (sum(range(193, 257)) + 64 * (4 + 64))
     assert abs(visible_flops(w) / 1e12 - 9.6e-6) < 0.05e-6          # the tiny configuration's figure
@@ -468,7 +468,7 @@ def test_visible_flops_match_hand_count_and_enumeration():
 def test_mass_pair_count_matches_enumeration():
     """The token-mass leg's work count (one exponential per visible (query row, query head, key of the query
     range)) against the oracle's explicit visible sets."""
-    import bench
+    from head_sparse_paged_b200.counts import mass_pairs
     w = synth.custom("ragged", [(1000, 300), (37, 37), (5, 0), (129, 1), (300, 300)], 8, 2, 64, 16,
                      [[(0, 0, 100), (1, 0, 0)], [(0, 50, 3), (0, 2, 1)], [(1, 0, 0), (0, 1, 1)],
                       [(0, 128, 1), (1, 0, 0)], [(0, 1000, 2), (0, 127, 129)]], seed=7)
@@ -477,4 +477,4 @@ def test_mass_pair_count_matches_enumeration():
         for kh in range(w.num_kv_heads):
             g, S, W = (int(x) for x in w.classes[0, b, kh])
             want += sum(int((orc.visible_keys(bool(g), S, W, i) >= L - Lq).sum()) for i in range(L - Lq, L))
-    assert bench.mass_pairs(w, 0) == w.group * want
+    assert mass_pairs(w, 0) == w.group * want
