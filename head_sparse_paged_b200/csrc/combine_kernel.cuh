@@ -4,9 +4,9 @@
 // chunk's softmax-weighted V sum normalised by its own row sum, and LSE_c, the natural-log sum of the
 // chunk's exponentials (-inf when the row saw no visible key in it). Exact attention over the union is
 //   LSE = log sum_c exp(LSE_c),   O = sum_c exp(LSE_c - LSE) O_c.
-// One pass per row merges the chunks online (running max, rescaled sum and accumulator), four chunks'
+// One pass per row merges the chunks online (running max, rescaled sum and accumulator), eight chunks'
 // loads in flight at a time; rows of records with few chunks get a warp each, rows of records with many
-// chunks a whole block whose eight per-warp results are merged in a fixed order. The order of the merge
+// chunks a whole block whose eight per-warp results (four loads in flight each) are merged in a fixed order. The order of the merge
 // depends only on the plan, never on which CTA ran which chunk. Each lane owns D/32 columns (coalesced).
 #pragma once
 #include <cuda_bf16.h>
@@ -43,18 +43,19 @@ struct CombineParams {
   int32_t* status;         // nullable
 };
 
-// Online merge of chunks c = c0, c0 + stride, ... into (m, wsum, acc): loads of four chunks are issued
-// together, the running max rescales what was accumulated so far when it grows.
-template <int V>
+// Online merge of chunks c = c0, c0 + stride, ... into (m, wsum, acc): the loads of NB chunks are issued
+// together (one round trip for a record of up to NB chunks), the running max rescales what was accumulated
+// so far when it grows.
+template <int V, int NB>
 __device__ __forceinline__ void merge_chunks(const float* part_o, const float* part_lse, int32_t part0, int32_t nsplit,
                                              int c0, int stride, int r, int lane, int D, float& m, float& wsum,
                                              float (&acc)[V]) {
   int c = c0;
-  for (; c < nsplit; c += 4 * stride) {
-    float lc[4];
-    float2 v[4][V / 2];
+  for (; c < nsplit; c += NB * stride) {
+    float lc[NB];
+    float2 v[NB][V / 2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < NB; ++u) {
       const int cc = c + u * stride;
       lc[u] = -INFINITY;
       if (cc < nsplit) {
@@ -66,7 +67,7 @@ __device__ __forceinline__ void merge_chunks(const float* part_o, const float* p
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < NB; ++u) {
       if (lc[u] == -INFINITY) continue;  // no visible key of this row in the chunk (or past the end)
       if (lc[u] > m) {
         const float f = (m == -INFINITY) ? 0.f : expf(m - lc[u]);
@@ -128,8 +129,10 @@ __global__ void __launch_bounds__(256) segpaged_combine_kernel(const CombinePara
     float m = -INFINITY, wsum = 0.f, acc[V];
 #pragma unroll
     for (int k = 0; k < V; ++k) acc[k] = 0.f;
-    if (active) merge_chunks<V>(p.part_o, p.part_lse, part0, nsplit, wide ? warp : 0, wide ? NW : 1, r, lane, D, m,
-                                wsum, acc);
+    if (active) {
+      if (wide) merge_chunks<V, 4>(p.part_o, p.part_lse, part0, nsplit, warp, NW, r, lane, D, m, wsum, acc);
+      else merge_chunks<V, 8>(p.part_o, p.part_lse, part0, nsplit, 0, 1, r, lane, D, m, wsum, acc);
+    }
     if (wide) {
       if (lane == 0) {
         s_m[warp] = m;
