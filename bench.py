@@ -652,30 +652,35 @@ def measure_mass(runner, args, world, device):
     ev = []
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        for li in runner.layers:
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            runner.token_mass(li)
-            b.record(stream)
-            runner.select_topk(li, k_per_seq, selected)
-            ev.append((li, a, b))
-    t1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(device.index if device.index is not None else 0, interval=0.01) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            for li in runner.layers:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                runner.token_mass(li)
+                b.record(stream)
+                runner.select_topk(li, k_per_seq, selected)
+                ev.append((li, a, b))
+        t1.record(stream)
+        torch.cuda.synchronize()
     runner.check_status()
     total_ms = t0.elapsed_time(t1)
     mass_ms = sum(a.elapsed_time(b) for _, a, b in ev)
     exps = sum(pairs[li] for li, _, _ in ev)
     peaks, _ = load_peaks()
-    clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
-    peak = MUFU_EX2_PER_CLK_SM * torch.cuda.get_device_properties(device).multi_processor_count * clk
+    clk_hz = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    peak = MUFU_EX2_PER_CLK_SM * torch.cuda.get_device_properties(device).multi_processor_count * clk_hz
     achieved = exps / (mass_ms * 1e-3)
+    ck = clk.summary()
+    # the same peak at the SM clock sampled during these launches (under the power cap the clock sits below max)
+    at_clock = peak * (ck["sm_mhz"] * 1e6 / clk_hz) if ck.get("sm_mhz") else None
     return {"kernel": "segpaged_mass_kernel (+ reduce)", "ms_per_layer": mass_ms / len(ev),
             "with_topk_ms_per_layer": total_ms / len(ev), "visible_pairs_per_step": sum(pairs.values()),
             "bound": "alu", "achieved": achieved / 1e9, "peak": peak / 1e9, "unit": "G exp2/s",
             "frac": achieved / peak, "peak_source": f"{MUFU_EX2_PER_CLK_SM} ex2/clk/SM x SMs x sm_max_mhz",
+            "frac_at_sampled_clock": achieved / at_clock if at_clock else None, "clocks": ck,
             "topk_frac": args.topk_frac}
 
 
@@ -746,9 +751,32 @@ def measure_rope_gather(runner, args, device, flops_layer, plain_prefill_ms_per_
             ev2.append((li, a, b))
     torch.cuda.synchronize()
     runner.check_status()
+    # the caller-level choice between the two (Runner.prefill_rope_auto), timed the same way
+    runner.frags = frags
+    try:
+        for _ in range(args.warmup):
+            for li in runner.layers:
+                runner.prefill_rope_auto(li, k_out)
+        torch.cuda.synchronize()
+        ev3, path = [], None
+        for _ in range(args.steps):
+            for li in runner.layers:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                path = runner.prefill_rope_auto(li, k_out)
+                b.record(stream)
+                ev3.append((li, a, b))
+        torch.cuda.synchronize()
+        runner.check_status()
+    finally:
+        runner.frags = None
     del k_out
     ms2 = sum(a.elapsed_time(b) for _, a, b in ev2)
+    ms3 = sum(a.elapsed_time(b) for _, a, b in ev3)
     return {"kernel": "segpaged_prefill_kernel<ROPE>", "fragment_tokens": args.fragment_tokens,
+            "auto_path": path, "auto_ms_per_layer": ms3 / len(ev3), "auto_tflops": flops / (ms3 * 1e-3) / 1e12,
+            "auto_time_vs_plain_prefill": (ms3 / args.steps) / plain_prefill_ms_per_step,
             "fragments": len(starts), "prefill_ms_per_layer": ms / len(ev),
             "tflops": flops / (ms * 1e-3) / 1e12, "time_vs_plain_prefill": per_step / plain_prefill_ms_per_step,
             "realign_then_prefill_ms_per_layer": ms2 / len(ev2),

@@ -244,9 +244,11 @@ __global__ void __launch_bounds__(512, 1)
         int go = 1;
         if (lane == 0) go = ptx::mbar_wait(&sh.unit_empty[slot], ((ring >> 1) & 1) ^ 1, abort, status, kStatusTimeout);
         if (!__shfl_sync(0xffffffffu, go, 0)) break;
-        // claim the next unit only once a ring slot is free, so no CTA sits on work it cannot start
+        // claim the next unit only once a ring slot is free, so no CTA sits on work it cannot start; the first
+        // unit of CTA i is unit i (the grid never exceeds the unit count), which takes the atomic off the
+        // start-up path, and later claims come from the counter, offset by the grid
         int32_t u = 0;
-        if (lane == 0) u = atomicAdd(p.counter, 1);
+        if (lane == 0) u = ring == 0 ? (int32_t)blockIdx.x : (int32_t)gridDim.x + atomicAdd(p.counter, 1);
         u = __shfl_sync(0xffffffffu, u, 0);
         const bool done = u >= p.num_units;
         int32_t* U = sh.unit[slot];

@@ -227,9 +227,12 @@ int64_t plan_units(const segpaged_dims* dims, const int32_t* ctx_len, const int3
   auto cost = [](const segpaged_unit& u) { return (int64_t)u.v[U_NTILES] * (u.v[U_HALF] ? 1 : 2); };
   // Split long units across CTAs when one unit alone would exceed a CTA's fair share of the work (short
   // query ranges, decode-like tiles). A unit longer than a target T is cut into near-equal chunks of at
-  // least 4 KV tiles (at most 256 chunks). T is chosen among one to four waves of the CTAs by simulating
-  // the longest-first schedule with a fixed per-record overhead (queries, pipeline fill, partial write),
-  // so a split is only as fine as the makespan rewards; ties keep the coarser split (less partial traffic).
+  // least 4 KV tiles (at most 256 chunks); each chunk writes a partial result that the combine launch merges.
+  // T is chosen by a cost model of the whole call, fitted to launches measured on this B200 (one cost unit, a KV
+  // tile of one query tile, is about 1 us of the launch): the longest-first schedule of the records over the
+  // CTAs with a fixed cost per record (claim, query load, pipeline ramp), plus the partial rows the chunks write
+  // and the combine merges, plus the combine launch itself. Candidates run from one to four waves of equal
+  // pieces up to no split at all, so short units are left whole when splitting them costs more than it saves.
   std::vector<segpaged_unit> groups;
   int32_t slots = 0;
   if (split_ctas > 0 && !out.empty()) {
@@ -241,36 +244,50 @@ int64_t plan_units(const segpaged_dims* dims, const int32_t* ctx_len, const int3
     if (longest * split_ctas > total) {
       auto chunk_of = [](const segpaged_unit& u, int64_t target) {
         const int32_t weight = u.v[U_HALF] ? 1 : 2;
-        int32_t chunk = (int32_t)std::max<int64_t>(4, ceil_div(target, weight));
+        int32_t chunk = (int32_t)std::max<int64_t>(4, std::min<int64_t>(INT32_MAX, ceil_div(target, weight)));
         return std::max<int32_t>(chunk, (int32_t)ceil_div(u.v[U_NTILES], kCombineMaxSplit));
       };
-      constexpr int64_t kRecordOverhead = 4;   // fixed cost of a record, in tile x query-tile units
-      int64_t best_target = 0, best_span = INT64_MAX;
-      for (int waves = 1; waves <= 4; ++waves) {
-        const int64_t target = ceil_div(total, (int64_t)waves * split_ctas);
+      constexpr double kRecordCost = 6.0;      // per record, in cost units
+      constexpr double kPartialRowCost = 3e-4; // per partial row (written by a chunk, read by the combine)
+      constexpr double kCombineCost = 4.0;     // the combine launch, when anything is split
+      auto model = [&](int64_t target) {
         std::vector<int64_t> items;
+        int64_t rows = 0;
         for (const auto& u : out) {
           const int32_t n = u.v[U_NTILES], chunk = chunk_of(u, target), weight = u.v[U_HALF] ? 1 : 2;
           if (n <= chunk) {
-            items.push_back(cost(u) + kRecordOverhead);
+            items.push_back(cost(u));
             continue;
           }
           const int32_t k = (int32_t)ceil_div(n, chunk);
-          for (int32_t c = 0; c < k; ++c) items.push_back((int64_t)(n / k + (c < n % k ? 1 : 0)) * weight + kRecordOverhead);
+          for (int32_t c = 0; c < k; ++c) items.push_back((int64_t)(n / k + (c < n % k ? 1 : 0)) * weight);
+          rows += (int64_t)k * u.v[U_NPOS] * G;
         }
         std::sort(items.begin(), items.end(), std::greater<int64_t>());
-        std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> load;
-        for (int32_t c = 0; c < split_ctas; ++c) load.push(0);
-        int64_t span = 0;
+        std::priority_queue<double, std::vector<double>, std::greater<double>> load;
+        for (int32_t c = 0; c < split_ctas; ++c) load.push(0.0);
+        double span = 0.0;
         for (int64_t it : items) {
-          const int64_t x = load.top() + it;
+          const double x = load.top() + (double)it + kRecordCost;
           load.pop();
           load.push(x);
           span = std::max(span, x);
         }
-        if (span < best_span) {
-          best_span = span;
-          best_target = target;
+        return span + (rows > 0 ? kCombineCost + kPartialRowCost * (double)rows : 0.0);
+      };
+      std::vector<int64_t> targets;
+      for (int waves = 4; waves >= 1; --waves) targets.push_back(ceil_div(total, (int64_t)waves * split_ctas));
+      for (int64_t t = targets.back(); t < longest;) {
+        t = std::max<int64_t>(t + 1, t * 5 / 4);
+        targets.push_back(std::min(t, longest));    // the last candidate splits nothing
+      }
+      int64_t best_target = longest;
+      double best_time = model(longest);
+      for (int64_t t : targets) {   // ties keep the coarser split (less partial traffic): candidates ascend
+        const double x = model(t);
+        if (x < best_time - 1e-9 || (x <= best_time + 1e-9 && t > best_target)) {
+          best_time = x;
+          best_target = t;
         }
       }
       std::vector<segpaged_unit> work;

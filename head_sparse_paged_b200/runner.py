@@ -222,6 +222,27 @@ class Runner:
         sp.segpaged_attn_prefill(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info,
                                  self.scale, st.o, st.lse, self.workspace, self.status, stream)
 
+    def rope_realign_preferred(self) -> bool:
+        """Which gather-time RoPE path the caller should take (see prefill_rope_auto): the re-alignment pass when
+        some (sequence, KV head) has more than one work unit, i.e. its query range spans more than 2 x 128 / G
+        positions, so that every K tile would be rotated once per unit that loads it."""
+        return rope_realign_preferred(self.w.q_lens, self.w.group)
+
+    def prefill_rope_auto(self, li, k_scratch, stream=None):
+        """Prefill with the fragments' RoPE re-alignment (self.frags) by the cheaper of the two exact paths:
+        segpaged_rope_realign of the layer's K pages into k_scratch (a second pool of the same shape) followed by
+        the plain prefill on it, when rope_realign_preferred(); else the gather-time kernel, which rotates each K
+        tile in shared memory as it lands. Both give bit-identical O and LSE."""
+        st = self.state[li]
+        if not self.rope_realign_preferred():
+            self.prefill(li, stream)
+            return "gather"
+        sp.segpaged_rope_realign(self.dims, self.cu_k_dev, self.ql_dev, st.cls_dev, st.table_dev, st.offs_dev,
+                                 *self.frags, self.k_pool, k_scratch, self.status, stream)
+        sp.segpaged_attn_prefill(self.dims, st.q, k_scratch, self.v_pool, st.table_dev, st.units_dev, st.info,
+                                 self.scale, st.o, st.lse, self.workspace, self.status, stream)
+        return "realign"
+
     def plan_mass(self, li):
         """Host planning of one layer's token-mass items."""
         st = self.state[li]
@@ -262,3 +283,10 @@ class Runner:
         s = int(self.status.item())
         if s:
             raise RuntimeError(f"device status word {s:#x}")
+
+
+def rope_realign_preferred(q_lens, group: int) -> bool:
+    """True when some sequence's query range spans more than one work unit (2 x 128 / G positions) per KV head:
+    each K tile is then loaded, and rotated at gather time, by several units, and one re-alignment pass over the
+    stored pages costs less."""
+    return max(q_lens, default=0) > 2 * (128 // group)

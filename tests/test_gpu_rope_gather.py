@@ -165,3 +165,18 @@ def test_realign_pass_then_plain_prefill_equals_gather_time_rope_bitwise(name):
                            w.page_size, st.table, st.offs, r.num_pages)
     used = ~np.isnan(kp[:, 0, 0])
     np.testing.assert_array_equal(k_out.float().cpu().numpy()[used], kp[used])
+
+
+def test_caller_level_rope_path_equals_gather_time_bitwise():
+    """Runner.prefill_rope_auto takes the re-alignment pass on a layer whose query range spans several units per
+    KV head, and returns the gather-time kernel's O and LSE bit for bit."""
+    w = SMALL["g2-p64"]()
+    fr = _fragments(w, np.random.default_rng(65), per_seq=6)
+    g = _run(w, frags=fr)
+    r = Runner(w, keep_dense=True, frags=fr, split_ctas=g.split_ctas)
+    k_out = torch.zeros_like(r.k_pool)
+    assert r.rope_realign_preferred()
+    assert r.prefill_rope_auto(0, k_out) == "realign"
+    torch.cuda.synchronize()
+    r.check_status()
+    assert torch.equal(r.state[0].o, g.state[0].o) and torch.equal(r.state[0].lse, g.state[0].lse)

@@ -478,3 +478,15 @@ def test_mass_pair_count_matches_enumeration():
             g, S, W = (int(x) for x in w.classes[0, b, kh])
             want += sum(int((orc.visible_keys(bool(g), S, W, i) >= L - Lq).sum()) for i in range(L - Lq, L))
     assert mass_pairs(w, 0) == w.group * want
+
+
+def test_rope_path_choice():
+    """The caller-level RoPE path: re-alignment pass when a (sequence, KV head) has more than one work unit of
+    2 x 128 / G positions, gather-time rotation otherwise."""
+    from head_sparse_paged_b200.runner import rope_realign_preferred
+    assert not rope_realign_preferred([16] * 32, 8)          # decode-like batch: one unit per head
+    assert not rope_realign_preferred([32, 5], 8)            # exactly one unit of 2 x 16 positions
+    assert rope_realign_preferred([33], 8)
+    assert rope_realign_preferred([4096], 1)                 # 43-layer workload: 16 units per head
+    assert not rope_realign_preferred([256], 1) and rope_realign_preferred([257], 1)
+    assert not rope_realign_preferred([], 4)
