@@ -422,6 +422,8 @@ __global__ void __launch_bounds__(kMassThreads, 1)
     }
   }
 
+  // every warp arrives at the block barrier converged, so each is counted once before tensor memory is freed
+  __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == C::MMA) {

@@ -42,6 +42,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "combine_kernel.cuh"
 #include "plan.h"
 #include "rope.cuh"
 #include "sm100_ptx.cuh"
@@ -88,7 +89,8 @@ struct PrefillParams {
   int32_t* status;       // nullable
   __nv_bfloat16* o;      // [total_q, Hq, D]
   float* lse;            // [Hq, total_q]
-  float* part_o;         // [partial slots][256 rows][D] fp32: O / l of one chunk of a split unit
+  float* part_o;         // [partial slots][D/4][256 rows] fp32 4-column groups (partial_o_index): O / l of one
+                         // chunk of a split unit
   float* part_lse;       // [partial slots][256 rows] fp32: LSE of that chunk (natural log)
   int32_t total_q, num_q_heads, num_pages, log2_group;
   int32_t num_partials;  // partial slots in part_o / part_lse
@@ -542,8 +544,8 @@ __global__ void __launch_bounds__(512, 1)
           // rows and slots outside the call are skipped here and reported by the softmax warps
           const bool store_row = pslot < u[U_NPOS] && qrow >= 0 && qrow < p.total_q && head >= 0 &&
                                  head < p.num_q_heads;
-          float* pdst = (part >= 0 && part < p.num_partials) ? p.part_o + ((int64_t)part * 256 + t * 128 + row) * D
-                                                             : nullptr;
+          const bool to_part = part >= 0 && part < p.num_partials;
+          float4* pdst = reinterpret_cast<float4*>(p.part_o);
           __nv_bfloat16* odst = (part < 0 && store_row) ? p.o + (qrow * p.num_q_heads + head) * D : nullptr;
 #pragma unroll 1
           for (int c = 0; c < D / 16; ++c) {
@@ -569,10 +571,11 @@ __global__ void __launch_bounds__(512, 1)
                 if (two_o) ptx::mbar_arrive(&sh.o_free[1]);
               }
             }
-            if (pdst) {
+            if (to_part) {   // 4-column groups 4c .. 4c + 3 of this row, coalesced over the warp's rows
 #pragma unroll
               for (int k = 0; k < 4; ++k)
-                reinterpret_cast<float4*>(pdst + c * 16)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                pdst[partial_o_index<D>(part, t * 128 + row, c * 4 + k)] =
+                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
             } else if (odst) {
               uint32_t w[8];
 #pragma unroll
@@ -1060,14 +1063,14 @@ __global__ void __launch_bounds__(512, 1)
         const bool empty = (m_run == -INFINITY) || !(l_run > 0.f);
         const float inv_l = empty ? 0.f : 1.0f / l_run;
         const int64_t prow = (int64_t)part * 256 + tile * 128 + row;
-        float* dst = p.part_o + prow * D;
+        float4* dst = reinterpret_cast<float4*>(p.part_o);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           load_o(c, r);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            reinterpret_cast<float4*>(dst + c * 32)[k] =
+          for (int k = 0; k < 8; ++k)   // 4-column groups 8c .. 8c + 7, coalesced over the warp's rows
+            dst[partial_o_index<D>(part, tile * 128 + row, c * 8 + k)] =
                 make_float4(__uint_as_float(r[4 * k]) * inv_l, __uint_as_float(r[4 * k + 1]) * inv_l,
                             __uint_as_float(r[4 * k + 2]) * inv_l, __uint_as_float(r[4 * k + 3]) * inv_l);
         }
@@ -1102,6 +1105,9 @@ __global__ void __launch_bounds__(512, 1)
   }
 
   // ------------------------------------------------------------------------------------ teardown
+  // Every warp arrives at the block barrier converged (the roles leave their loops after lane-0-only
+  // arrivals), so each warp is counted once and tensor memory is released only after every role is done.
+  __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 9) {

@@ -453,11 +453,12 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 template <int D>
 int launch_combine(const CombineParams& c, cudaStream_t st) {
   if (c.num_groups <= 0) return SEGPAGED_OK;
-  // records x row blocks (as many as the widest record needs), as a programmatic dependent launch: its
+  // records x row blocks of 32 rows (as many as the widest record needs) x 8 column ranges (used by records
+  // of more than 16 chunks), as a programmatic dependent launch: its
   // blocks are scheduled while the prefill's last CTAs finish and wait in the kernel for that grid's
   // completion
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)std::min<int64_t>(c.num_groups, 65535), (unsigned)c.row_blocks);
+  cfg.gridDim = dim3((unsigned)std::min<int64_t>(c.num_groups, 65535), (unsigned)c.row_blocks, 8);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
@@ -577,7 +578,7 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   c.log2_group = p.log2_group;
   c.status = status;
   const int64_t rb = info->combine_row_blocks;
-  c.row_blocks = (rb > 0 && rb < kCombineRows) ? (int32_t)rb : kCombineRows;
+  c.row_blocks = (rb > 0 && rb < kCombineRows / kCombineBlockRows) ? (int32_t)rb : kCombineRows / kCombineBlockRows;
   return D == 128 ? launch_combine<128>(c, st) : launch_combine<64>(c, st);
 }
 }  // namespace

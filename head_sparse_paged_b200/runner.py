@@ -290,3 +290,31 @@ def rope_realign_preferred(q_lens, group: int) -> bool:
     each K tile is then loaded, and rotated at gather time, by several units, and one re-alignment pass over the
     stored pages costs less."""
     return max(q_lens, default=0) > 2 * (128 // group)
+
+
+def main(argv=None):
+    """Sets one or more layers of a workload up and runs their prefill launches back to back (for a profiler:
+    `python -m head_sparse_paged_b200.runner dsv4-flash --layers 3 --launches 2`). Layers draw their own dense
+    K/V, which is freed after the build, so only the pool, the queries and the outputs stay on the device."""
+    import argparse
+    ap = argparse.ArgumentParser(description=main.__doc__)
+    ap.add_argument("workload")
+    ap.add_argument("--layers", default="0", help="comma-separated layer indices")
+    ap.add_argument("--launches", type=int, default=2, help="prefill launches per layer")
+    args = ap.parse_args(argv)
+    w = synth.get(args.workload)
+    layers = [int(x) for x in args.layers.split(",")]
+    r = Runner(w, layers=layers)
+    torch.cuda.synchronize()
+    for _ in range(args.launches):
+        for li in layers:
+            r.prefill(li)
+    torch.cuda.synchronize()
+    r.check_status()
+    print(f"{w.name}: layers {layers}, {args.launches} prefill launches each, pool {r.num_pages} pages, "
+          f"{torch.cuda.max_memory_allocated() / 1e9:.2f} GB peak device memory")
+    return 0
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())

@@ -96,9 +96,8 @@ typedef struct {
  * tiles alternate between both softmax warpgroups, which merge their two partial results at the end;
  * == num_units: the unused second query buffer also serves as one more K/V slot); results are correct
  * for any value below num_units, but the variants round differently. combine_row_blocks sizes the
- * combine launch: the most thread blocks one combine record needs (one per row for a record of more than
- * 16 chunks, else one per 8 rows), 0 for "unknown" (256 per record). A value below what the plan needs
- * leaves rows unmerged and sets SEGPAGED_STATUS_UNIT.
+ * combine launch: the most blocks of 32 rows one combine record needs, 0 for "unknown" (8, a whole
+ * record). A value below what the plan needs leaves rows unmerged and sets SEGPAGED_STATUS_UNIT.
  * The last six fields record the call the plan was made for: its records address query rows
  * [0, total_q), query heads [0, num_q_heads) and page-table entries [0, page_table_len) (the planner's
  * page_table_offs[B*Hkv]). The prefill entry points return SEGPAGED_ERR_DIMS before any launch when the

@@ -144,12 +144,12 @@ def _units_cover_exactly(w_seqs, Hq, Hkv, D, P, classes, split_ctas=0):
     assert not chunks and len(slots) == info["num_partials"]
     assert np.all(seen == 1)
     # the combine grid reaches the last valid row of every record: row of position p, head h is
-    # (p // (128/G)) * 128 + (p % (128/G)) * G + h; a block per row above 16 chunks, else per 8 rows
+    # (p // (128/G)) * 128 + (p % (128/G)) * G + h; a block per 32 rows
     npt = 128 // G
     need = 0
     for grp in groups:
         last = max((p // npt) * 128 + (p % npt) * G + G - 1 for p in range(int(grp[U_NPOS]))) + 1
-        need = max(need, last if grp[U_NSPLIT] > 16 else -(-last // 8))
+        need = max(need, -(-last // 32))
     assert info["combine_row_blocks"] == need
     assert info["num_half_units"] == sum(int(u[U_HALF]) for u in units)
     return units
