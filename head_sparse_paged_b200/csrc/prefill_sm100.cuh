@@ -15,9 +15,8 @@
 //               lazy O rescale (only when the running max grows by more than 2^8), exp2 on the MUFU
 //               unit (one pair in eight on the FMA pipe by a cubic, beside it), row sum and scaling in packed
 //               f32x2 arithmetic, P written back to TMEM as bf16 over
-//               S and published in two halves of 64 keys. At the end of a unit they write the row's
-//               LSE = ln 2 * (m + log2 l) and hand the row's O scale (1 / l) to the epilogue warpgroup, then
-//               go straight on to the next unit; with ROPE they do the O epilogue themselves.
+//               S and published in two halves of 64 keys, and the epilogue (O / l -> bf16,
+//               LSE = ln 2 * (m + log2 l)).
 //   warp 8      producer (whole warp: page-table lookups; lane 0: barriers and TMA): claims units, TMA-loads both Q tiles (3-D map over [rows, Hq, D], box
 //               64 x G x 128/G) and, for every 128-key tile, the K and V pages (3-D map over
 //               [pages, P, D], coordinate = physical page id) into 128B-swizzled shared-memory slots.
@@ -28,11 +27,7 @@
 //               S_t(j) its O_t is stable and can be rescaled.
 //   warps 10-11 idle, or when appending (fused append-and-attend) writing the new keys and values of the
 //               unit's query positions into their pool pages.
-//   warps 12-15 without ROPE: the epilogue. Once a unit's last P V has landed they read O out of TMEM,
-//               scale it (merging the two accumulators of a shared half unit) and store it (bf16 O, or the
-//               fp32 partial of a split chunk), releasing the accumulator as soon as it is read, so the
-//               softmax warps never wait on the O read-out and stores between units.
-//               With ROPE: the gather-time RoPE re-alignment. They rotate each K tile in shared
+//   warps 12-15 only with ROPE: the gather-time RoPE re-alignment. They rotate each K tile in shared
 //               memory once it lands (keys of reused fragments, from their original to their actual
 //               positions, per sequence fragment) and only then release it to the MMA warp.
 // Every wait is bounded: on a timeout the CTA raises its abort flag, reports SEGPAGED_STATUS_TIMEOUT,
@@ -64,19 +59,18 @@ struct PrefillCfg {
   static constexpr int NSLOT = (D == 128) ? 5 : 10;
   static constexpr int PPT = BN / P;             // pages per KV tile
   static constexpr int SMEM_BYTES = 2 * Q_BYTES + NSLOT * TILE_BYTES + 1024;
-  static constexpr bool EPI = !ROPE;             // warps 12-15 run the O epilogue (else they rotate K)
-  static constexpr int THREADS = 512;            // a fourth warpgroup: the epilogue, or with ROPE the K rotation
+  static constexpr int THREADS = ROPE ? 512 : 384;   // ROPE: a fourth warpgroup rotates K tiles
   static constexpr uint32_t TMEM_COLS = 512;     // S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D)
   static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t IDESC_O = ptx::idesc_bf16_f32(128, D, 0, 1);
-  // Register split (setmaxnreg) within the 512 x 128 = 65536 registers the block is launched with:
-  // 256 softmax threads x 192 + 128 producer/MMA threads x 64 + 128 epilogue (or RoPE) threads x 64 = 65536.
-  // (Fewer for the producer and MMA warps made them spill; the softmax code fits in 192.)
-  static constexpr int REGS_SOFTMAX = 192;
-  static constexpr int REGS_OTHER = 64;
-  static constexpr int REGS_FOURTH = 64;
-  static constexpr int LAUNCH_REGS = 128;
-  static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER + 128 * REGS_FOURTH <= THREADS * LAUNCH_REGS,
+  // Register split (setmaxnreg): 256 softmax threads x 208 + 128 other threads x 80 = 63488, within the
+  // 384 x 168 = 64512 registers the block is launched with; with ROPE 256 x 192 + 128 x 64 (producer,
+  // MMA) + 128 x 64 (RoPE warpgroup) = 65536 = 512 x 128.
+  static constexpr int REGS_SOFTMAX = ROPE ? 192 : 208;
+  static constexpr int REGS_OTHER = ROPE ? 64 : 80;
+  static constexpr int REGS_ROPE = 64;
+  static constexpr int LAUNCH_REGS = ROPE ? 128 : 168;
+  static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER + (ROPE ? 128 * REGS_ROPE : 0) <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch budget");
 };
 
@@ -119,13 +113,8 @@ struct PrefillShared {
   uint64_t k_rot[11];      // ROPE: K tile of tile count n rotated (ring over n % NSLOT), ready for the MMA
   __align__(16) int32_t unit[2][U_NFIELDS];
   int32_t frag_start[ROPE ? kRopeSmemFragments : 1];   // ROPE: the current unit's sequence fragment starts
-  // Without ROPE: the O scale of row r of accumulator t at fin[t * 128 + r], handed from the softmax warpgroups to
-  // the epilogue warpgroup once per unit (fin_full: 8 softmax warps; fin_empty: 4 epilogue warps). On a shared
-  // half unit warpgroup 1 first leaves its running max and sum there (fin[r], fin[128 + r], ml_full) for
-  // warpgroup 0's merge. With ROPE: the merge hand-off alone (ml_full / ml_empty, at fin[2r], fin[2r + 1]).
-  float fin[256];
-  uint64_t ml_full, ml_empty;
-  uint64_t fin_full, fin_empty;
+  float ml[256];              // shared half units: warpgroup 1's running max and sum per row, for the merge
+  uint64_t ml_full, ml_empty; // ... written by warpgroup 1 (4 warps), read by warpgroup 0 (4 warps)
   uint32_t tmem_base;
   int abort;
 };
@@ -148,7 +137,7 @@ constexpr int kModePlain = 0, kModeRope = 1, kModeAppend = 2;
 // HALF (chosen per launch): 0 -- every unit has rows in both query tiles; 1 -- the plan has half units;
 // 2 -- every unit is a half unit.
 template <int D, int P, int MODE, int HALF>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
                             const __grid_constant__ CUtensorMap tm_vn, const PrefillParams p) {
@@ -177,8 +166,8 @@ __global__ void __launch_bounds__(512, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sh.unit_full[i], 1);
-      // MMA warp + 8 softmax warps + 4 RoPE or epilogue warps (+ 2 append warps)
-      ptx::mbar_init(&sh.unit_empty[i], APPEND ? 15 : 13);
+      // MMA warp + 8 softmax warps (+ 4 RoPE warps, or + 2 append warps)
+      ptx::mbar_init(&sh.unit_empty[i], ROPE ? 13 : (APPEND ? 11 : 9));
       ptx::mbar_init(&sh.s_full[i], 1);
       ptx::mbar_init(&sh.p_half[i], 4);
       ptx::mbar_init(&sh.p_full[i], 4);
@@ -190,8 +179,6 @@ __global__ void __launch_bounds__(512, 1)
     ptx::mbar_init(&sh.mma_drain, 1);
     ptx::mbar_init(&sh.ml_full, 4);
     ptx::mbar_init(&sh.ml_empty, 4);
-    ptx::mbar_init(&sh.fin_full, 8);
-    ptx::mbar_init(&sh.fin_empty, 4);
     for (int i = 0; i < NSLOT; ++i) {
       ptx::mbar_init(&sh.kv_full[i], 1);
       ptx::mbar_init(&sh.kv_empty[i], 1);
@@ -233,7 +220,7 @@ __global__ void __launch_bounds__(512, 1)
 
   if (warp >= 8) {
     if (warp < 12) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
-    else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_FOURTH));
+    else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_ROPE));
     if (warp == 8) {
       // ---------------------------------------------------------------------------- producer
       // The whole warp walks the schedule; lane 0 does the barrier and TMA work, and the 32 lanes fetch
@@ -496,103 +483,7 @@ __global__ void __launch_bounds__(512, 1)
       ptx::umma_commit(leader, &sh.mma_drain);
       ptx::mbar_wait(&sh.mma_drain, 0, nullptr, status, kStatusTimeout);
       __syncwarp();
-    } else if (C::EPI && warp >= 12) {
-      // ------------------------------------------------------------------------------ epilogue
-      // Walks the schedule like the MMA warp. Per unit: the O scales the softmax warps handed over, then per
-      // output tile (one for a half unit, two otherwise) the accumulator once its last P V has landed, read in
-      // chunks of 16 columns (both accumulators of a shared half unit, merged), scaled and stored as bf16 O or
-      // as the fp32 partial of a split chunk. The accumulator is released to the MMA warp after its last chunk
-      // is read, before the last stores.
-      const int quarter = warp & 3;
-      const int row = quarter * 32 + lane;
-      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-      uint32_t o0cnt = 0, o1cnt = 0, fcnt = 0;
-      auto ewait = [&](uint64_t* bar, uint32_t parity) -> bool {
-        return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kStatusTimeout));
-      };
-      for (uint32_t ring = 0;; ++ring) {
-        const int slot = ring & 1;
-        if (!ewait(&sh.unit_full[slot], (ring >> 1) & 1)) break;
-        const int32_t* u = sh.unit[slot];
-        const int32_t ntiles = u[U_NTILES];
-        if (ntiles < 0) {
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
-          break;
-        }
-        const bool is_half = ALL_HALF || u[U_HALF] != 0;
-        const bool two_o = SHARED_HALF && is_half && ntiles >= 2;
-        if (!ewait(&sh.fin_full, fcnt & 1)) break;
-        ++fcnt;
-        const float sc0 = sh.fin[row], sc1 = sh.fin[128 + row];
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.fin_empty);
-        const int32_t part = u[U_PART];
-        bool ok = true;
-        for (int t = 0; t < (is_half ? 1 : 2); ++t) {
-          if (!ewait(&sh.o_full[t], (t == 0 ? o0cnt : o1cnt) & 1) || (two_o && !ewait(&sh.o_full[1], o1cnt & 1))) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-          const uint32_t obuf = tmem + 256 + t * D + lane_off;
-          const uint32_t obuf1 = tmem + 256 + D + lane_off;
-          const float s0 = t == 0 ? sc0 : sc1;
-          const int32_t pslot = t * npos + (row >> p.log2_group);
-          const int32_t head = u[U_KVH] * G + (row & (G - 1));
-          const int64_t qrow = (int64_t)u[U_QROW] + pslot;
-          // rows and slots outside the call are skipped here and reported by the softmax warps
-          const bool store_row = pslot < u[U_NPOS] && qrow >= 0 && qrow < p.total_q && head >= 0 &&
-                                 head < p.num_q_heads;
-          const bool to_part = part >= 0 && part < p.num_partials;
-          float4* pdst = reinterpret_cast<float4*>(p.part_o);
-          __nv_bfloat16* odst = (part < 0 && store_row) ? p.o + (qrow * p.num_q_heads + head) * D : nullptr;
-#pragma unroll 1
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t r[16];
-            float v[16];
-            ptx::tmem_ld16(obuf + c * 16, r);
-            if (two_o) {
-              uint32_t r1[16];
-              ptx::tmem_ld16(obuf1 + c * 16, r1);
-              ptx::tmem_ld_wait();
-#pragma unroll
-              for (int k = 0; k < 16; ++k) v[k] = __fmaf_rn(sc1, __uint_as_float(r1[k]), s0 * __uint_as_float(r[k]));
-            } else {
-              ptx::tmem_ld_wait();
-#pragma unroll
-              for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]) * s0;
-            }
-            if (c == D / 16 - 1) {   // the accumulator(s) are read: the next unit's first P V may overwrite them
-              ptx::tc_fence_before();
-              __syncwarp();
-              if (lane == 0) {
-                ptx::mbar_arrive(&sh.o_free[t]);
-                if (two_o) ptx::mbar_arrive(&sh.o_free[1]);
-              }
-            }
-            if (to_part) {   // 4-column groups 4c .. 4c + 3 of this row, coalesced over the warp's rows
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                pdst[partial_o_index<D>(part, t * 128 + row, c * 4 + k)] =
-                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-            } else if (odst) {
-              uint32_t w[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k) w[k] = ptx::pack_bf16x2(v[2 * k], v[2 * k + 1]);
-              reinterpret_cast<uint4*>(odst + c * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              reinterpret_cast<uint4*>(odst + c * 16)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            }
-          }
-          if (t == 0) ++o0cnt;
-          else ++o1cnt;
-          if (two_o) ++o1cnt;
-        }
-        if (!ok) break;
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
-      }
-    } else if (APPEND && warp >= 10 && warp < 12) {
+    } else if (APPEND && warp >= 10) {
       // ------------------------------------------------------------------------------ append
       // Warps 10-11 write the new keys and values of the unit's own query positions into their pool pages
       // (the positions of a (sequence, KV head) are split among its units, so every new row is written
@@ -744,7 +635,6 @@ __global__ void __launch_bounds__(512, 1)
     // completed uses of O0 and O1 (phases of o_full[0], o_full[1]) and of the half-unit hand-off, counted
     // by both warpgroups over every unit
     uint32_t o0cnt = 0, o1cnt = 0, mlcnt = 0;
-    uint32_t fcnt = 0;   // hand-offs to the epilogue warpgroup (phases of fin_full / fin_empty)
     // The tcgen05.ld/st below are warp-collective, so every wait's outcome is made warp-uniform.
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, status, kStatusTimeout));
@@ -760,12 +650,6 @@ __global__ void __launch_bounds__(512, 1)
       const bool shared_half = SHARED_HALF && is_half;           // both warpgroups on query tile 0
       const bool two_o = shared_half && ntiles >= 2;             // ... and O1 holds warpgroup 1's share
       if (ntiles < 0 || (tile == 1 && is_half && !SHARED_HALF)) {   // end of schedule, or no rows for us
-        if (C::EPI && ntiles >= 0) {   // every softmax warp takes part in every unit's hand-off cycle
-          if (!wwait(&sh.fin_empty, (fcnt & 1) ^ 1)) break;
-          ++fcnt;
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&sh.fin_full);
-        }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.unit_empty[slot]);
         if (ntiles < 0) break;
@@ -932,73 +816,14 @@ __global__ void __launch_bounds__(512, 1)
       }
       if (!ok) break;
 
-      if constexpr (C::EPI) {
-        // ---------------------------------------------------------------- hand-off to the epilogue
-        // The row's LSE is written here; its O scale goes to the epilogue warpgroup, which reads O once the
-        // unit's last P V has landed. These warps go on to the next unit at once.
-        if (!wwait(&sh.fin_empty, (fcnt & 1) ^ 1)) break;   // the previous unit's scales have been read
-        ++fcnt;
-        if (shared_half && tile == 1) {
-          if (two_o) {   // running max and sum of this warpgroup's KV tiles, for warpgroup 0's merge
-            sh.fin[row] = m_run;
-            sh.fin[128 + row] = l_run;
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&sh.ml_full);
-            ++mlcnt;
-          }
-          __syncwarp();
-          if (lane == 0) {
-            ptx::mbar_arrive(&sh.fin_full);
-            ptx::mbar_arrive(&sh.unit_empty[slot]);
-          }
-          continue;
-        }
-        // weights of the two accumulators: (1, 0) unless this is a shared half unit with two shares
-        float a0 = 1.f, a1 = 0.f;
-        if (two_o) {
-          if (!wwait(&sh.ml_full, mlcnt & 1)) break;
-          ++mlcnt;
-          const float m1 = sh.fin[row], l1 = sh.fin[128 + row];
-          const float M = fmaxf(m_run, m1);
-          a0 = (m_run == -INFINITY) ? 0.f : ptx::ex2(m_run - M);
-          a1 = (m1 == -INFINITY) ? 0.f : ptx::ex2(m1 - M);
-          l_run = a0 * l_run + a1 * l1;
-          m_run = M;
-        }
-        // a row that saw no visible key (only possible in a chunk of a split unit) gets O = 0, LSE = -inf
-        const bool empty = (m_run == -INFINITY) || !(l_run > 0.f);
-        const float inv_l = empty ? 0.f : 1.0f / l_run;
-        const float lse = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
-        sh.fin[tile * 128 + row] = a0 * inv_l;   // tile is 0 on a shared half unit
-        if (two_o) sh.fin[128 + row] = a1 * inv_l;
-        const int32_t part = u[U_PART];
-        if (part >= 0) {
-          if (part < p.num_partials) p.part_lse[(int64_t)part * 256 + tile * 128 + row] = lse;
-          else if (status && quarter == 0 && lane == 0) atomicOr(status, kStatusUnit);
-        } else if (valid_row) {
-          const int64_t qrow = (int64_t)u[U_QROW] + pslot;
-          if (qrow >= 0 && qrow < p.total_q && head >= 0 && head < p.num_q_heads)
-            p.lse[(int64_t)head * p.total_q + qrow] = lse;
-          else if (status)
-            atomicOr(status, kStatusUnit);
-        }
-        __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(&sh.fin_full);
-          ptx::mbar_arrive(&sh.unit_empty[slot]);
-        }
-        continue;
-      }
-
       // ------------------------------------------------------------------------------ epilogue
-      // (ROPE: the softmax warps read O out themselves; warps 12-15 rotate K tiles)
       if (shared_half && tile == 1) {
         // hand the running max and sum of warpgroup 1's KV tiles to warpgroup 0, which merges
         if (two_o) {
           // the previous hand-off has been read
           if (!wwait(&sh.ml_empty, (mlcnt & 1) ^ 1)) break;
-          sh.fin[2 * row] = m_run;
-          sh.fin[2 * row + 1] = l_run;
+          sh.ml[2 * row] = m_run;
+          sh.ml[2 * row + 1] = l_run;
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&sh.ml_full);
           ++o1cnt;
@@ -1013,7 +838,7 @@ __global__ void __launch_bounds__(512, 1)
       float a0 = 1.f, a1 = 0.f;
       if (two_o) {
         if (!wwait(&sh.ml_full, mlcnt & 1) || !wwait(&sh.o_full[1], o1cnt & 1)) break;
-        const float m1 = sh.fin[2 * row], l1 = sh.fin[2 * row + 1];
+        const float m1 = sh.ml[2 * row], l1 = sh.ml[2 * row + 1];
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sh.ml_empty);
         const float M = fmaxf(m_run, m1);
@@ -1051,30 +876,29 @@ __global__ void __launch_bounds__(512, 1)
         if (two_o) ++mlcnt;
       };
       const int32_t part = u[U_PART];
-      if (part >= p.num_partials) {
-        // a record that names a partial slot the workspace does not have (not from this call's plan)
-        if (status && quarter == 0 && lane == 0) atomicOr(status, kStatusUnit);
-        release();
-        continue;
-      }
       if (part >= 0) {
         // one chunk of a split unit: O / l in fp32 and the chunk's LSE, for the combine pass; a row that
-        // saw no visible key in this chunk writes O = 0 and LSE = -inf
+        // saw no visible key in this chunk writes O = 0 and LSE = -inf. A slot the workspace does not have
+        // (a record from another plan) is skipped and reported.
         const bool empty = (m_run == -INFINITY) || !(l_run > 0.f);
         const float inv_l = empty ? 0.f : 1.0f / l_run;
-        const int64_t prow = (int64_t)part * 256 + tile * 128 + row;
+        const bool slot_ok = part < p.num_partials;
+        if (!slot_ok && status && quarter == 0 && lane == 0) atomicOr(status, kStatusUnit);
+        const int32_t prow = tile * 128 + row;
         float4* dst = reinterpret_cast<float4*>(p.part_o);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           load_o(c, r);
+          if (slot_ok) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k)   // 4-column groups 8c .. 8c + 7, coalesced over the warp's rows
-            dst[partial_o_index<D>(part, tile * 128 + row, c * 8 + k)] =
-                make_float4(__uint_as_float(r[4 * k]) * inv_l, __uint_as_float(r[4 * k + 1]) * inv_l,
-                            __uint_as_float(r[4 * k + 2]) * inv_l, __uint_as_float(r[4 * k + 3]) * inv_l);
+            for (int k = 0; k < 8; ++k)   // 4-column groups 8c .. 8c + 7, coalesced over the warp's rows
+              dst[partial_o_index<D>(part, prow, c * 8 + k)] =
+                  make_float4(__uint_as_float(r[4 * k]) * inv_l, __uint_as_float(r[4 * k + 1]) * inv_l,
+                              __uint_as_float(r[4 * k + 2]) * inv_l, __uint_as_float(r[4 * k + 3]) * inv_l);
+          }
         }
-        p.part_lse[prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        if (slot_ok) p.part_lse[(int64_t)part * 256 + prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
         release();
         continue;
       }
