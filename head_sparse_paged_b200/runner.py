@@ -114,6 +114,9 @@ class Runner:
         if self.frags is not None:
             self.rope = None          # the pools keep the keys as drawn; prefill re-aligns them per fragment
         self.scale = 1.0 / math.sqrt(D)
+        # per layer: the build and plain-prefill calls with their arguments marshalled once (PreparedCall), so a
+        # step's host overhead per call is one ctypes call; rebuilt when the plan's shape or the workspace changes
+        self._prep_build, self._prep_prefill = {}, {}
         for li in self.layers:
             self._setup_layer(li)
 
@@ -205,8 +208,16 @@ class Runner:
                 lo, hi = int(ck[b + 1]) - w.q_lens[b], int(ck[b + 1])
                 k[lo:hi] = -3.0 * k[lo:hi] + 1.0
                 v[lo:hi] = 0.5 * v[lo:hi] - 2.0
-        sp.segpaged_build(self.dims, k, v, self.cu_k_dev, self.ql_dev, st.cls_dev, st.table_dev, st.offs_dev, self.rope,
-                          self.k_pool, self.v_pool, self.status, stream)
+        if self.append or self._tmp_dense is not None:       # per-call inputs: marshal them each time
+            sp.segpaged_build(self.dims, k, v, self.cu_k_dev, self.ql_dev, st.cls_dev, st.table_dev, st.offs_dev,
+                              self.rope, self.k_pool, self.v_pool, self.status, stream)
+            return
+        call = self._prep_build.get(li)
+        if call is None:
+            call = self._prep_build[li] = sp.prepare_build(self.dims, k, v, self.cu_k_dev, self.ql_dev, st.cls_dev,
+                                                            st.table_dev, st.offs_dev, self.rope, self.k_pool,
+                                                            self.v_pool, self.status)
+        call(stream)
 
     def prefill(self, li, stream=None):
         st = self.state[li]
@@ -219,8 +230,13 @@ class Runner:
             sp.segpaged_attn_prefill_rope(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info,
                                           self.scale, *self.frags, st.o, st.lse, self.workspace, self.status, stream)
             return
-        sp.segpaged_attn_prefill(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info,
-                                 self.scale, st.o, st.lse, self.workspace, self.status, stream)
+        key = (id(self.workspace), tuple(st.info.values()))
+        cached = self._prep_prefill.get(li)
+        if cached is None or cached[0] != key:
+            cached = self._prep_prefill[li] = (key, sp.prepare_attn_prefill(
+                self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info, self.scale, st.o,
+                st.lse, self.workspace, self.status))
+        cached[1](stream)
 
     def rope_realign_preferred(self) -> bool:
         """Which gather-time RoPE path the caller should take (see prefill_rope_auto): the re-alignment pass when

@@ -179,18 +179,26 @@ def segpaged_rope_cos_sin(theta: float, deltas, head_dim: int) -> np.ndarray:
     return out
 
 
+def prepare_build(dims: Dims, k_dense, v_dense, cu_seqlens_k, q_len, cls, page_table, page_table_offs, rope_cos_sin,
+                  k_pool, v_pool, status=None) -> PreparedCall:
+    """segpaged_build with its arguments checked and marshalled once (see PreparedCall)."""
+    bf = torch.bfloat16
+    d = dims.c()
+    args = (ctypes.byref(d), _dev(k_dense, bf, "k_dense"), _dev(v_dense, bf, "v_dense"),
+            _dev(cu_seqlens_k, torch.int32, "cu_seqlens_k"), _dev(q_len, torch.int32, "q_len"),
+            _dev(cls, torch.int32, "cls"), _dev(page_table, torch.int32, "page_table"),
+            _dev(page_table_offs, torch.int32, "page_table_offs"), _dev(rope_cos_sin, torch.float32, "rope_cos_sin"),
+            _dev(k_pool, bf, "k_pool"), _dev(v_pool, bf, "v_pool"), _dev(status, torch.int32, "status"))
+    return PreparedCall(_lib.segpaged_build, "segpaged_build", args,
+                        (d, k_dense, v_dense, cu_seqlens_k, q_len, cls, page_table, page_table_offs, rope_cos_sin,
+                         k_pool, v_pool, status))
+
+
 def segpaged_build(dims: Dims, k_dense, v_dense, cu_seqlens_k, q_len, cls, page_table, page_table_offs,
                    rope_cos_sin, k_pool, v_pool, status=None, stream=None):
     """Scatter dense K/V [sum L, Hkv, D] (bf16, CUDA) into k_pool/v_pool [num_pages, P, D]."""
-    bf = torch.bfloat16
-    r = _lib.segpaged_build(ctypes.byref(dims.c()), _dev(k_dense, bf, "k_dense"), _dev(v_dense, bf, "v_dense"),
-                            _dev(cu_seqlens_k, torch.int32, "cu_seqlens_k"), _dev(q_len, torch.int32, "q_len"),
-                            _dev(cls, torch.int32, "cls"), _dev(page_table, torch.int32, "page_table"),
-                            _dev(page_table_offs, torch.int32, "page_table_offs"),
-                            _dev(rope_cos_sin, torch.float32, "rope_cos_sin"), _dev(k_pool, bf, "k_pool"),
-                            _dev(v_pool, bf, "v_pool"), _dev(status, torch.int32, "status"), _stream(stream))
-    if r < 0:
-        raise SegPagedError(r, "segpaged_build")
+    prepare_build(dims, k_dense, v_dense, cu_seqlens_k, q_len, cls, page_table, page_table_offs, rope_cos_sin, k_pool,
+                  v_pool, status)(stream)
 
 
 def _info(d: dict) -> _PlanInfo:
@@ -232,19 +240,42 @@ def segpaged_prefill_workspace_bytes(dims: Dims, info: dict) -> int:
     return int(_lib.segpaged_prefill_workspace_bytes(ctypes.byref(dims.c()), ctypes.byref(_info(info))))
 
 
+class PreparedCall:
+    """A C-ABI call whose arguments were checked and marshalled once, for callers that repeat it (a serving loop
+    runs the same layer's prefill every step). The tensors it was prepared with must stay allocated, with the same
+    shape, dtype, device and storage, while it is used; their contents may change between calls. Calling it passes
+    the given CUDA stream (default: the current one) and raises SegPagedError on a negative return code."""
+
+    __slots__ = ("_fn", "_name", "_args", "_keep")
+
+    def __init__(self, fn, name: str, args: tuple, keep: tuple):
+        self._fn, self._name, self._args, self._keep = fn, name, args, keep
+
+    def __call__(self, stream=None):
+        r = self._fn(*self._args, _stream(stream))
+        if r < 0:
+            raise SegPagedError(r, self._name)
+
+
+def prepare_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, plan, info: dict, softmax_scale, o, lse, workspace,
+                         status=None) -> PreparedCall:
+    """segpaged_attn_prefill with its arguments checked and marshalled once (see PreparedCall)."""
+    bf = torch.bfloat16
+    d, inf = dims.c(), _info(info)
+    args = (ctypes.byref(d), _dev(q, bf, "q"), int(q.shape[0]), _dev(k_pool, bf, "k_pool"), _dev(v_pool, bf, "v_pool"),
+            _dev(page_table, torch.int32, "page_table"), int(page_table.numel()), _dev(plan, torch.int32, "plan"),
+            ctypes.byref(inf), float(softmax_scale), _dev(o, bf, "o"), _dev(lse, torch.float32, "lse"),
+            _dev(workspace, None, "workspace"), int(workspace.numel() * workspace.element_size()),
+            _dev(status, torch.int32, "status"))
+    return PreparedCall(_lib.segpaged_attn_prefill, "segpaged_attn_prefill", args,
+                        (d, inf, q, k_pool, v_pool, page_table, plan, o, lse, workspace, status))
+
+
 def segpaged_attn_prefill(dims: Dims, q, k_pool, v_pool, page_table, plan, info: dict, softmax_scale, o, lse, workspace,
                           status=None, stream=None):
     """O [total_q, Hq, D] bf16 and LSE [Hq, total_q] float32, written in place (CUDA tensors).
     plan: the plan's records on the device; info: the dict segpaged_prefill_plan returned."""
-    bf = torch.bfloat16
-    r = _lib.segpaged_attn_prefill(ctypes.byref(dims.c()), _dev(q, bf, "q"), int(q.shape[0]), _dev(k_pool, bf, "k_pool"),
-                                   _dev(v_pool, bf, "v_pool"), _dev(page_table, torch.int32, "page_table"),
-                                   int(page_table.numel()), _dev(plan, torch.int32, "plan"), ctypes.byref(_info(info)),
-                                   float(softmax_scale), _dev(o, bf, "o"), _dev(lse, torch.float32, "lse"),
-                                   _dev(workspace, None, "workspace"), int(workspace.numel() * workspace.element_size()),
-                                   _dev(status, torch.int32, "status"), _stream(stream))
-    if r < 0:
-        raise SegPagedError(r, "segpaged_attn_prefill")
+    prepare_attn_prefill(dims, q, k_pool, v_pool, page_table, plan, info, softmax_scale, o, lse, workspace, status)(stream)
 
 
 def segpaged_attn_prefill_append(dims: Dims, q, k_new, v_new, k_pool, v_pool, page_table, plan, info: dict,
