@@ -63,6 +63,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-dense", action="store_true",
                     help="skip the dense-layout baseline (explicit mask) on an all-global and a mixed layer")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="issue each prefill call directly instead of replaying its CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle sample (per step in --impl reference)")
     return ap.parse_args(argv)
@@ -415,7 +417,8 @@ def run_ours(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = rank_workload(args.workload, rank)
-    runner = Runner(w, device=device, keep_dense=True, shared_dense=(w.layers > 1), mass=not args.no_mass)
+    runner = Runner(w, device=device, keep_dense=True, shared_dense=(w.layers > 1), mass=not args.no_mass,
+                    graphs=not args.no_graphs)
     torch.cuda.synchronize()
     runner.check_status()
     flops_layer = {li: visible_flops(w, [li]) for li in runner.layers}
@@ -539,6 +542,8 @@ def run_ours(args, rank, world, local):
         "append": append,
         "gpu_launches": args.steps * sum(launches_layer.values()),
         "gpu_launches_note": "per layer and step: build scatter, prefill, and the combine where the plan splits units",
+        "prefill_submission": "direct C-ABI call" if args.no_graphs else
+                              "CUDA graph of the C-ABI call per layer (captured in warm-up, replayed every step)",
         "clocks": clocks,
     }
     print(json.dumps(line))
@@ -572,7 +577,7 @@ def measure_workloads(args, device, names):
     out = {}
     for name in names:
         w = synth.get(name)
-        r = Runner(w, device=device)
+        r = Runner(w, device=device, graphs=not args.no_graphs)
         torch.cuda.synchronize()
         r.check_status()
         stream = torch.cuda.current_stream()

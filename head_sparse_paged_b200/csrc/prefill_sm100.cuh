@@ -235,9 +235,12 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         if (!__shfl_sync(0xffffffffu, go, 0)) break;
         // claim the next unit only once a ring slot is free, so no CTA sits on work it cannot start; the first
         // unit of CTA i is unit i (the grid never exceeds the unit count), which takes the atomic off the
-        // start-up path, and later claims come from the counter, offset by the grid
+        // start-up path, and later claims come from the counter, offset by the grid. A launch with one unit
+        // per CTA never touches the counter (the host does not clear it for such a launch).
         int32_t u = 0;
-        if (lane == 0) u = ring == 0 ? (int32_t)blockIdx.x : (int32_t)gridDim.x + atomicAdd(p.counter, 1);
+        if (lane == 0)
+          u = ring == 0 ? (int32_t)blockIdx.x
+                        : ((int32_t)gridDim.x >= p.num_units ? p.num_units : (int32_t)gridDim.x + atomicAdd(p.counter, 1));
         u = __shfl_sync(0xffffffffu, u, 0);
         const bool done = u >= p.num_units;
         int32_t* U = sh.unit[slot];

@@ -519,7 +519,9 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   const int sms = device_sm_count(dev);
   if (sms <= 0) return SEGPAGED_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), st) != cudaSuccess) return SEGPAGED_ERR_CUDA;
+  const int grid = (int)std::min<int64_t>(num_units, sms);
+  // the work counter is read only when some CTA claims a second unit
+  if (num_units > grid && cudaMemsetAsync(workspace, 0, sizeof(int32_t), st) != cudaSuccess) return SEGPAGED_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   PrefillParams p;
   p.page_table = page_table;
@@ -548,7 +550,6 @@ int attn_prefill(const segpaged_dims* dims, const void* q, int32_t total_q, cons
   p.v_new = static_cast<const __nv_bfloat16*>(v_new);
   p.k_pool = static_cast<__nv_bfloat16*>(const_cast<void*>(k_pool));
   p.v_pool = static_cast<__nv_bfloat16*>(const_cast<void*>(v_pool));
-  const int grid = (int)std::min<int64_t>(num_units, sms);
   rc = SEGPAGED_ERR_DIMS;
 #define SEGPAGED_LAUNCH(DD, PP)                                                   \
   if (D == DD && P == PP)                                                          \
@@ -625,7 +626,8 @@ extern "C" int segpaged_attn_prefill_rope(const segpaged_dims* dims, const void*
 // cannot provide the work-unit list and the work-counter workspace that segpaged_attn_prefill needs.
 // For them, both live in one file-scope device array below. Every GPU that loads this library holds
 // it (2 MiB) until the process exits. All calls on a device share it and it keeps the last call's
-// contents, so the counter is cleared on every call; calls whose work overlaps on the GPU race on it.
+// contents, so the counter is cleared by every call that reads it; calls whose work overlaps on the
+// GPU race on it.
 // ------------------------------------------------------------------------------------------------
 namespace {
 constexpr int64_t kNoAllocMaxUnits = 16384;   // the most work units one call accepts
@@ -686,7 +688,7 @@ extern "C" int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const vo
   if (cudaMemcpyAsync(units_dev, units_host, sizeof(segpaged_unit) * (size_t)num_units, cudaMemcpyHostToDevice, st) !=
       cudaSuccess)
     return SEGPAGED_ERR_CUDA;
-  // The work counter (word 0) is zeroed on the stream by segpaged_attn_prefill before its launch.
+  // The work counter (word 0) is zeroed on the stream before a launch that claims units from it.
   segpaged_plan_info info;
   info.num_units = num_units;
   info.num_groups = 0;

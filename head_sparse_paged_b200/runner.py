@@ -57,10 +57,14 @@ class Runner:
     append: fused append-and-attend -- the build writes only the rows before each query range (the query
     rows' pool slots get unrelated values) and each prefill writes the query rows' keys/values into the pool
     while attending over them.
+    graphs: run each layer's plain prefill call as a CUDA graph, captured once per plan shape, so that the
+    call's launches (counter clear, prefill, combine) reach the GPU as one submission and its short launches
+    do not wait on the host between them. The graph reads the same buffers as the call it was captured from,
+    so every replay sees the plan, queries and pages the step has just written.
     """
 
     def __init__(self, w: synth.Workload, device="cuda", layers=None, keep_dense=False, page_seed_offset=0,
-                 shared_dense=False, split_ctas=None, mass=False, frags=None, append=False):
+                 shared_dense=False, split_ctas=None, mass=False, frags=None, append=False, graphs=False):
         self.w = w
         self.device = torch.device(device)
         # long units are split across CTAs when one alone exceeds a CTA's share (short query ranges)
@@ -117,6 +121,7 @@ class Runner:
         # per layer: the build and plain-prefill calls with their arguments marshalled once (PreparedCall), so a
         # step's host overhead per call is one ctypes call; rebuilt when the plan's shape or the workspace changes
         self._prep_build, self._prep_prefill = {}, {}
+        self.graphs = graphs
         for li in self.layers:
             self._setup_layer(li)
 
@@ -233,10 +238,22 @@ class Runner:
         key = (id(self.workspace), tuple(st.info.values()))
         cached = self._prep_prefill.get(li)
         if cached is None or cached[0] != key:
-            cached = self._prep_prefill[li] = (key, sp.prepare_attn_prefill(
-                self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev, st.info, self.scale, st.o,
-                st.lse, self.workspace, self.status))
-        cached[1](stream)
+            call = sp.prepare_attn_prefill(self.dims, st.q, self.k_pool, self.v_pool, st.table_dev, st.units_dev,
+                                           st.info, self.scale, st.o, st.lse, self.workspace, self.status)
+            if not self.graphs:
+                cached = self._prep_prefill[li] = (key, call, None)
+            else:
+                call(stream)     # this call's prefill, issued directly; the graph serves the calls after it
+                self._prep_prefill[li] = (key, call, capture_graph(call, self.device))
+                return
+        _, call, graph = cached
+        if graph is None:
+            call(stream)
+        elif stream is None:
+            graph.replay()
+        else:
+            with torch.cuda.stream(stream):
+                graph.replay()
 
     def rope_realign_preferred(self) -> bool:
         """Which gather-time RoPE path the caller should take (see prefill_rope_auto): the re-alignment pass when
@@ -299,6 +316,17 @@ class Runner:
         s = int(self.status.item())
         if s:
             raise RuntimeError(f"device status word {s:#x}")
+
+
+def capture_graph(call, device) -> torch.cuda.CUDAGraph:
+    """A CUDA graph of one prepared C-ABI call that has already run once on `device` (the library configures
+    a kernel on its first launch on a device, which must not happen inside a capture). Capturing launches
+    nothing; replaying the graph repeats the call's launches with the same arguments."""
+    with torch.cuda.device(device):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call(None)
+    return g
 
 
 def rope_realign_preferred(q_lens, group: int) -> bool:

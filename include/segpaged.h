@@ -198,8 +198,8 @@ size_t segpaged_prefill_workspace_bytes(const segpaged_dims* dims, const segpage
 
 /*
  * EXECUTE: causal attention of every query head over its own ragged paged KV (one persistent
- * kernel launch, preceded by a 4-byte memset of the workspace; for split plans followed by one
- * combine launch).
+ * kernel launch, preceded by a 4-byte memset of the workspace's work counter when the plan has more
+ * units than the GPU has SMs; for split plans followed by one combine launch).
  *   q (dev) [total_q, Hq, D] bf16.  k_pool, v_pool (dev) [num_pages, P, D] bf16.
  *   page_table (dev, int32) [page_table_len].
  *   plan (dev) [info->num_units + info->num_groups] records from segpaged_prefill_plan; info (host).
@@ -301,7 +301,7 @@ int segpaged_attn_prefill_rope(const segpaged_dims* dims, const void* q, int32_t
  * until the process exits; it holds at most 16384 units (more return SEGPAGED_ERR_CAPACITY). The
  * first call on a device looks up the array's device address; make that first call before any
  * stream capture. Every call on a device shares the array and it keeps the last call's contents (the
- * work counter is cleared on every call): calls whose work overlaps on the GPU race, so serialise
+ * work counter is cleared by every call that reads it): calls whose work overlaps on the GPU race, so serialise
  * them (one stream, or events). Allocates no memory.
  */
 int segpaged_attn_prefill_noalloc(const segpaged_dims* dims, const void* q, int32_t total_q, const void* k_pool,

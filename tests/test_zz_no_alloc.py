@@ -7,7 +7,9 @@ counter live in a static device array of the library instead of caller-provided 
 It runs the same kernel variant on the same plan as segpaged_attn_prefill, so its O and LSE must be the
 workspace entry point's bit for bit, and within the parity tolerances of the fp64 oracle on every row.
 Calls run back to back, the later ones on a plan with fewer units than the array still holds from the
-earlier ones, so a unit left behind by an earlier call would show. This file is collected last.
+earlier ones, so a unit left behind by an earlier call would show. The first plan has more units than
+the GPU has SMs, so its CTAs claim units from the array's work counter, which the call clears; the
+others have one unit per CTA and leave the counter alone. This file is collected last.
 """
 import numpy as np
 import pytest
@@ -23,8 +25,18 @@ from gpu_common import compare, full_problem, oracle_dense
 pytestmark = pytest.mark.gpu
 
 
+# 160 half units (80 sequences x 2 KV heads, 20-64 query rows each): more units than SMs
+MANY = [(200 + (53 * i) % 190, 20 + (7 * i) % 45) for i in range(80)]
+
+
+def _workload(name):
+    if name == "many-units":
+        return synth.custom(name, MANY, 4, 2, 128, 16, [[(1, 0, 0), (0, 16, 64)]] * len(MANY), seed=31)
+    return synth.get(name)
+
+
 def _setup(name):
-    w = synth.get(name)
+    w = _workload(name)
     r = Runner(w, split_ctas=0, keep_dense=True)   # the allocation-free entry point takes plans without split units
     r.step()
     torch.cuda.synchronize()
@@ -38,10 +50,12 @@ def _setup(name):
 
 
 def test_noalloc_prefill_matches_workspace_entry_point_and_oracle():
-    cases = {name: _setup(name) for name in ("mistral-7b", "tiny")}
-    assert len(cases["tiny"][1].state[0].units) < len(cases["mistral-7b"][1].state[0].units)
-    # two calls on the larger plan, then two on the smaller one, over the array the larger plan filled
-    for name in ("mistral-7b", "mistral-7b", "tiny", "tiny"):
+    cases = {name: _setup(name) for name in ("many-units", "mistral-7b", "tiny")}
+    units = {name: len(c[1].state[0].units) for name, c in cases.items()}
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert units["tiny"] < units["mistral-7b"] < sms < units["many-units"], units
+    # calls on ever smaller plans, each over the array the larger plans before it filled
+    for name in ("many-units", "many-units", "mistral-7b", "mistral-7b", "tiny", "tiny"):
         w, r, o_ws, lse_ws, o_ref, lse_ref = cases[name]
         st = r.state[0]
         o = torch.full_like(st.o, float("nan"))
