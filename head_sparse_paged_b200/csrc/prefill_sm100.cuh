@@ -852,15 +852,18 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       }
       const uint32_t obuf1 = tmem + 256 + D + lane_off;   // O1, merged into O0's rows
       ptx::tc_fence_after();
-      // O chunk c of this warpgroup's rows, merged with O1 for a shared half unit
-      auto load_o = [&](int c, uint32_t (&r)[32]) {
-        ptx::tmem_ld32(obuf + c * 32, r);
+      // O columns [64 h, 64 h + 64) of this warpgroup's rows (two loads, one wait), merged with O1 for a shared
+      // half unit
+      auto load_o = [&](int h, uint32_t (&r)[64]) {
+        ptx::tmem_ld32(obuf + h * 64, r);
+        ptx::tmem_ld32(obuf + h * 64 + 32, r + 32);
         if (two_o) {
-          uint32_t r1[32];
-          ptx::tmem_ld32(obuf1 + c * 32, r1);
+          uint32_t r1[64];
+          ptx::tmem_ld32(obuf1 + h * 64, r1);
+          ptx::tmem_ld32(obuf1 + h * 64 + 32, r1 + 32);
           ptx::tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
+          for (int k = 0; k < 64; ++k)
             r[k] = __float_as_uint(__fmaf_rn(a1, __uint_as_float(r1[k]), a0 * __uint_as_float(r[k])));
         } else {
           ptx::tmem_ld_wait();
@@ -890,13 +893,13 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         const int32_t prow = tile * 128 + row;
         float4* dst = reinterpret_cast<float4*>(p.part_o);
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          load_o(c, r);
+        for (int h = 0; h < D / 64; ++h) {
+          uint32_t r[64];
+          load_o(h, r);
           if (slot_ok) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k)   // 4-column groups 8c .. 8c + 7, coalesced over the warp's rows
-              dst[partial_o_index<D>(part, prow, c * 8 + k)] =
+            for (int k = 0; k < 16; ++k)   // 4-column groups 16h .. 16h + 15, coalesced over the warp's rows
+              dst[partial_o_index<D>(part, prow, h * 16 + k)] =
                   make_float4(__uint_as_float(r[4 * k]) * inv_l, __uint_as_float(r[4 * k + 1]) * inv_l,
                               __uint_as_float(r[4 * k + 2]) * inv_l, __uint_as_float(r[4 * k + 3]) * inv_l);
           }
@@ -912,18 +915,25 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
       if (valid_row && !in_range && status) atomicOr(status, kStatusUnit);
       const bool store_row = valid_row && in_range;
       __nv_bfloat16* orow = p.o + (qrow * p.num_q_heads + head) * D;
+      // 32-byte stores when O is 32-byte aligned (every row then is: rows are D x 2 bytes apart)
+      const bool v8 = (reinterpret_cast<uintptr_t>(p.o) & 31) == 0;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        load_o(c, r);
-        uint32_t w[16];
+      for (int h = 0; h < D / 64; ++h) {
+        uint32_t r[64];
+        load_o(h, r);
+        uint32_t w[32];
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
+        for (int k = 0; k < 32; ++k)
           w[k] = ptx::pack_bf16x2(__uint_as_float(r[2 * k]) * inv_l, __uint_as_float(r[2 * k + 1]) * inv_l);
         if (store_row) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          if (v8) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            for (int k = 0; k < 4; ++k) ptx::st_global_v8(orow + h * 64 + k * 16, w + 8 * k);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow + h * 64);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
         }
       }
       if (store_row) p.lse[(int64_t)head * p.total_q + qrow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;

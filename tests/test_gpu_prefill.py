@@ -153,6 +153,27 @@ def test_prefill_is_deterministic_across_calls():
     assert torch.equal(o1, r.state[0].o) and torch.equal(l1, r.state[0].lse)
 
 
+@pytest.mark.parametrize("name", ["varlen-p16-g4", "mha-d64-p128"])
+def test_prefill_output_only_16_byte_aligned(name):
+    """O at an address that is 16- but not 32-byte aligned takes the epilogue's 16-byte stores; the result must be
+    the 32-byte-store path's bit for bit."""
+    from head_sparse_paged_b200 import segpaged as sp
+    w = SMALL[name]()
+    r = _run(w)
+    st = r.state[0]
+    buf = torch.full((st.o.numel() + 32,), float("nan"), dtype=torch.bfloat16, device=st.o.device)
+    base = (-(buf.data_ptr() // 2)) % 16                  # elements to the next 32-byte boundary
+    o = buf[base + 8: base + 8 + st.o.numel()].view(st.o.shape)
+    assert o.data_ptr() % 32 == 16
+    lse = torch.full_like(st.lse, float("nan"))
+    sp.segpaged_attn_prefill(r.dims, st.q, r.k_pool, r.v_pool, st.table_dev, st.units_dev, st.info, r.scale, o, lse,
+                             r.workspace, r.status)
+    torch.cuda.synchronize()
+    r.check_status()
+    assert st.o.data_ptr() % 32 == 0
+    assert torch.equal(o, st.o) and torch.equal(lse, st.lse)
+
+
 FULL = {
     "llama-3.3-70b": lambda: (synth.llama_70b(), [0]),
     "llama-3.3-70b-2-globals": lambda: (synth.llama_70b(globals_per_seq=2), [0]),
