@@ -459,10 +459,11 @@ def run_ours(args, rank, world, local):
     value = world * flops_step * args.steps / (ms_total * 1e-3) / 1e12
     achieved = sum(flops_layer[li] * len(prefill_ms[li]) for li in prefill_ms) / (prefill_total_ms * 1e-3) / 1e12
     peaks, src = load_peaks()
-    # A kernel timed inside a long run (or one that hit the power cap) is held to the sustained GEMM peak,
-    # a short burst at full clocks to the burst peak.
+    # A kernel timed inside a long run (or one whose clock the power cap held down) is held to the sustained GEMM
+    # peak, a short burst at full clocks to the burst peak.
     clocks = clk.summary()
-    sustained = ms_total >= 1000.0 or "sw_power_cap" in (clocks.get("reasons") or [])
+    sustained = ms_total >= 1000.0 or ("sw_power_cap" in (clocks.get("reasons") or []) and
+                                       (clocks.get("sm_mhz") or 0) < (clocks.get("sm_max_mhz") or 0))
     tf_name = "bf16_tflops_sustained" if sustained and "bf16_tflops_sustained" in peaks else "bf16_tflops"
     peak_tf = float(peaks[tf_name])
     peak_bw = float(peaks.get("hbm_gbs"))
@@ -568,7 +569,7 @@ def measure_workloads(args, device, names):
     set up through the same C ABI and timed like the headline's kernel: CUDA events around each launch (the
     prefill, and the combine where the plan splits units), W warm-up launches, then max(K, 30) timed ones, with
     the SM clock sampled every 10 ms. The fraction is taken against the burst GEMM peak, or the sustained one when
-    the power cap was active during the launches."""
+    the power cap held the median SM clock below its maximum during the launches."""
     import torch
     from head_sparse_paged_b200 import synth
     from head_sparse_paged_b200.counts import visible_flops
@@ -599,8 +600,10 @@ def measure_workloads(args, device, names):
         flops = visible_flops(w, [0])
         nbytes = r.state[0].stored_bytes + w.total_q * w.num_q_heads * (w.head_dim * 2 * 2 + 4)
         ck = clk.summary()
-        # held to the sustained GEMM peak when the power cap was active during these launches, else to the burst
-        capped = "sw_power_cap" in (ck.get("reasons") or [])
+        # held to the sustained GEMM peak when the power cap held the clock down during these launches (median SM
+        # clock below the maximum), else to the burst peak
+        capped = "sw_power_cap" in (ck.get("reasons") or []) and \
+            (ck.get("sm_mhz") or 0) < (ck.get("sm_max_mhz") or 0)
         tf_name = "bf16_tflops_sustained" if capped and "bf16_tflops_sustained" in peaks else "bf16_tflops"
         rl = _roofline(w, flops, nbytes, ms, peaks, tf_name, src)
         out[name] = {"prefill_ms": ms, "visible_tflop": flops / 1e12, "tflops": flops / (ms * 1e-3) / 1e12,

@@ -112,9 +112,6 @@ __global__ void __launch_bounds__(256) segpaged_combine_kernel(const CombinePara
   constexpr int GW = D / 32;      // 4-column groups per warp (D / 4 groups over 8 warps)
   __shared__ float s_m[NW][32], s_sum[NW][32];
   __shared__ float s_acc[NW][4 * GW][32];
-  // Launched as a programmatic dependent of the prefill: wait until that grid has completed and its
-  // partial results are visible.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = 1 << p.log2_group;
   const int npos_tile = 128 >> p.log2_group;

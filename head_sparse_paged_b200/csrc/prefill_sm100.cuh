@@ -207,9 +207,6 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
     for (int x = threadIdx.x; x < NSLOT * C::TILE_BYTES / 16; x += blockDim.x)
       reinterpret_cast<uint4*>(sKV)[x] = make_uint4(0, 0, 0, 0);
   }
-  // The combine launch that may follow this one (split plans) can be scheduled as SMs free up; it waits
-  // for this grid's completion before reading anything (programmatic dependent launch).
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();

@@ -1,9 +1,8 @@
 """The runner's CUDA-graph submission of the prefill call (Runner(graphs=True)), through the C ABI.
 
 A graph replays the launches of one segpaged_attn_prefill call -- the work-counter clear when the plan has more
-units than SMs, the persistent prefill kernel, and the combine kernel (a programmatic dependent launch) for split
-plans -- with the arguments of the call it was captured from. Its O and LSE must be the direct call's bit for bit,
-step after step, while the step re-plans, re-uploads the plan and re-builds the pool into the same buffers; and on
+units than SMs, the persistent prefill kernel, and the combine kernel for split plans -- with the arguments of
+the call it was captured from. Its O and LSE must be the direct call's bit for bit, step after step, while the step re-plans, re-uploads the plan and re-builds the pool into the same buffers; and on
 the smallest case every row must also match the fp64 oracle.
 """
 import numpy as np
