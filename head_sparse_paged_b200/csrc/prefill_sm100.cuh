@@ -698,6 +698,38 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
             need_mask = true;
           }
         }
+        // The row's visible columns of the tile as four 32-bit words, also worked out before S is ready: per
+        // page at most two column ranges (the sink part and the causal window part; one for a global head), each
+        // clipped to the page and, appending, to the pool or new-K/V side of q0.
+        uint32_t mw[4] = {0u, 0u, 0u, 0u};
+        if (need_mask) {
+          const int32_t wlo = W > i_pos ? 0 : i_pos - W + 1;   // first key of the window (key > i_pos - W)
+#pragma unroll
+          for (int c = 0; c < C::PPT; ++c) {
+            if (lp[c] < 0) continue;
+            const int32_t j0 = lp[c] * P;
+            int32_t lo = 0, hi = i_pos - j0 + 1;                // causal: key <= i_pos
+            if (APPEND) {
+              if (fresh) lo = max(lo, splitq - j0);
+              else hi = min(hi, splitq - j0);
+            }
+            int32_t a1 = lo, b1 = hi, a2 = 0, b2 = 0;
+            if (!is_global) {
+              b1 = min(hi, S - j0);                             // sink: key < S
+              a2 = max(lo, wlo - j0);
+              b2 = hi;
+            }
+            a1 = max(a1, 0) + c * P;
+            b1 = min(b1, P) + c * P;
+            a2 = max(a2, 0) + c * P;
+            b2 = min(b2, P) + c * P;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if ((k + 1) * 32 <= c * P || k * 32 >= (c + 1) * P) continue;   // compile-time: the page's words
+              mw[k] |= range_bits(a1 - 32 * k, b1 - 32 * k) | range_bits(a2 - 32 * k, b2 - 32 * k);
+            }
+          }
+        }
         if (!wwait(&sh.s_full[tile], scount & 1)) { ok = false; break; }
         ++scount;
         ptx::tc_fence_after();
@@ -716,17 +748,9 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
           if (h == 1) ptx::tmem_ld_wait();
           if (need_mask) {
 #pragma unroll
-            for (int c = 0; c < C::PPT; ++c) {
-              const int32_t base = lp[c] * P;
-#pragma unroll
-              for (int r = 0; r < P; ++r) {
-                const int col = c * P + r;               // compile-time: columns outside this half skip
-                if (col < h * 64 || col >= h * 64 + 64) continue;
-                const int32_t jj = base + r;
-                const bool vis = lp[c] >= 0 && jj <= i_pos && (is_global || jj < S || jj > i_pos - W) &&
-                                 (!APPEND || (fresh ? jj >= splitq : jj < splitq));
-                if (!vis) s[col] = -INFINITY;
-              }
+            for (int k = 0; k < 64; ++k) {
+              const int col = h * 64 + k;                // compile-time word and bit
+              if (!((mw[col >> 5] >> (col & 31)) & 1u)) s[col] = -INFINITY;
             }
           }
 #pragma unroll

@@ -257,6 +257,13 @@ __device__ __forceinline__ uint64_t exp2_cubic_pair(uint64_t x2) {
                  __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
 
+// Bits [lo, hi) of a 32-bit word (lo and hi clipped to [0, 32]; empty when hi <= lo).
+__device__ __forceinline__ uint32_t range_bits(int32_t lo, int32_t hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 32);
+  return hi > lo ? (uint32_t)((1ull << hi) - (1ull << lo)) : 0u;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
