@@ -355,15 +355,20 @@ __global__ void __launch_bounds__(kMassThreads, 1)
       for (int32_t t = 0; t < nt; ++t, ++qi, ++si) {
         const int s = qi % C::NQ, b = si % C::NWG;
         if (b != wg) continue;
+        // The query tile's positions [pa, pb] and which of them see key j, worked out before the logits are
+        // ready: positions j .. j + W - 1 for a key of a local head past its sink, j .. pb otherwise. As tile
+        // columns (G per position) that is one range, kept as bits for the edge pairs.
+        const int32_t pa = q0 + (t0 + t) * npos, pb = pa + npos - 1;
+        const bool none = j > pb || (!is_global && j >= S && j <= pa - W);
+        const bool all = j <= pa && (is_global || j < S || j > pb - W);
+        const int32_t vlo = max(j, pa);
+        const int32_t vhi = (is_global || j < S || W > pb - j) ? pb : j + W - 1;
+        const int32_t clo = (vlo - pa) << p.log2_group, chi = (vhi - pa + 1) << p.log2_group;
         if (!wwait(&sh.s_full[b], (si / C::NWG) & 1) || !wwait(&sh.q_full[s], (qi / C::NQ) & 1)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        // The query tile's positions [pa, pb]; which of them see key j.
-        const int32_t pa = q0 + (t0 + t) * npos, pb = pa + npos - 1;
-        const bool none = j > pb || (!is_global && j >= S && j <= pa - W);
-        const bool all = j <= pa && (is_global || j < S || j > pb - W);
         const float* nl = s_nlse + s * 128;
         const uint32_t sbuf = tmem + b * 128 + lane_off;
         uint64_t acc[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -384,11 +389,11 @@ __global__ void __launch_bounds__(kMassThreads, 1)
           if (!all) {
             // edge pair: logits of rows that cannot see key j drop out (masked before the exponentials,
             // so the exponential loop below has no per-element branch)
+            const uint32_t mw[2] = {range_bits(clo - half * 64, chi - half * 64),
+                                    range_bits(clo - half * 64 - 32, chi - half * 64 - 32)};
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-              const int32_t i = pa + ((half * 64 + c) >> p.log2_group);
-              if (!(j <= i && (is_global || j < S || j > i - W))) v[c] = -INFINITY;
-            }
+            for (int c = 0; c < 64; ++c)
+              if (!((mw[c >> 5] >> (c & 31)) & 1u)) v[c] = -INFINITY;
           }
 #pragma unroll
           for (int c = 0; c < 64; c += 4) {
