@@ -162,6 +162,40 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
   volatile int* abort = &sh.abort;
   int32_t* status = p.status;
 
+  // Physical page id of list position 32 * batch + lane of unit U (-1 past its list; 0, and a status bit, for a
+  // table index or page id outside the call's arrays).
+  auto fetch_pid = [&](const int32_t* U, int32_t batch) -> int32_t {
+    const int32_t x = (batch << 5) + lane;
+    const int64_t toff = U[U_TOFF];
+    int32_t pid = -1;
+    if (x < U[U_AN] + U[U_BN]) {
+      const int32_t idx = unit_table_index(U, x);
+      pid = 0;
+      if (idx < 0 || idx >= U[U_TOTAL] || toff + idx < 0 || toff + idx >= p.page_table_len) {
+        if (status) atomicOr(status, kStatusUnit);
+      } else {
+        pid = p.page_table[toff + idx];
+        if (pid < 0 || pid >= p.num_pages) {
+          if (status) atomicOr(status, kStatusPageId);
+          pid = 0;
+        }
+      }
+    }
+    return pid;
+  };
+  // The producer's first unit is unit blockIdx.x (the grid never exceeds the unit count). Its descriptor and the
+  // page ids of its first 32 list positions are fetched now, so those global-memory round trips overlap the
+  // block's set-up instead of delaying the first query and K/V loads.
+  int32_t pre_batch = -1, pre_pid = -1;
+  if (warp == 8) {
+    int32_t* U0 = sh.unit[0];
+    if (lane < U_NFIELDS / 4)
+      reinterpret_cast<int4*>(U0)[lane] = reinterpret_cast<const int4*>(p.units + (int64_t)blockIdx.x * U_NFIELDS)[lane];
+    __syncwarp();
+    pre_batch = (U0[U_T0] * C::PPT) >> 5;
+    pre_pid = fetch_pid(U0, pre_batch);
+  }
+
   // ---------------------------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -243,7 +277,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
         int32_t* U = sh.unit[slot];
         if (done) {
           if (lane == 0) U[U_NTILES] = -1;
-        } else if (lane < U_NFIELDS / 4) {
+        } else if (ring > 0 && lane < U_NFIELDS / 4) {    // ring 0: fetched before the set-up
           reinterpret_cast<int4*>(U)[lane] = reinterpret_cast<const int4*>(p.units + (int64_t)u * U_NFIELDS)[lane];
         }
         __syncwarp();
@@ -267,14 +301,13 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
           }
         }
         if (!__shfl_sync(0xffffffffu, go, 0)) break;
-        const int32_t npages = U[U_AN] + U[U_BN];
         const int32_t t0 = U[U_T0];
         const int32_t ntiles = U[U_NTILES];
-        const int64_t toff = U[U_TOFF];
         const int32_t noldt = U[U_NOLDT], new0 = U[U_NEW0], nnew = U[U_NNEW];
         const int32_t kvh = U[U_KVH], newrow0 = U[U_CUQ] - U[U_SPLITQ];   // new-K/V row of key position 0
         if (nnew > 0 && !APPEND && lane == 0 && status) atomicOr(status, kStatusUnit);   // append plan, plain call
-        int32_t batch = -1, my_pid = -1;   // page id of list position 32 * batch + lane (-1: none)
+        int32_t batch = ring == 0 ? pre_batch : -1;   // my_pid: page id of list position 32 * batch + lane
+        int32_t my_pid = ring == 0 ? pre_pid : -1;
         int ok = 1;
         for (int32_t j = t0; j < t0 + ntiles && ok; ++j) {
           int32_t pages[C::PPT];             // physical page ids (pool tiles) or logical pages (new-page tiles)
@@ -284,21 +317,7 @@ __global__ void __launch_bounds__(MODE == kModeRope ? 512 : 384, 1)
             const int32_t x0 = j * C::PPT;     // a tile's PPT positions never straddle a batch of 32
             if ((x0 >> 5) != batch) {
               batch = x0 >> 5;
-              const int32_t x = (batch << 5) + lane;
-              my_pid = -1;
-              if (x < npages) {
-                const int32_t idx = unit_table_index(U, x);
-                my_pid = 0;
-                if (idx < 0 || idx >= U[U_TOTAL] || toff + idx < 0 || toff + idx >= p.page_table_len) {
-                  if (status) atomicOr(status, kStatusUnit);
-                } else {
-                  my_pid = p.page_table[toff + idx];
-                  if (my_pid < 0 || my_pid >= p.num_pages) {
-                    if (status) atomicOr(status, kStatusPageId);
-                    my_pid = 0;
-                  }
-                }
-              }
+              my_pid = fetch_pid(U, batch);
             }
 #pragma unroll
             for (int c = 0; c < C::PPT; ++c) {
