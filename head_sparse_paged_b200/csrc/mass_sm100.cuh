@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kMassThreads, 1)
         const bool all = j <= pa && (is_global || j < S || j > pb - W);
         const int32_t vlo = max(j, pa);
         const int32_t vhi = (is_global || j < S || W > pb - j) ? pb : j + W - 1;
-        const int32_t clo = (vlo - pa) << p.log2_group, chi = (vhi - pa + 1) << p.log2_group;
+        const int32_t clo = (vlo - pa) * G, chi = (vhi - pa + 1) * G;     // chi < clo: nothing visible
         if (!wwait(&sh.s_full[b], (si / C::NWG) & 1) || !wwait(&sh.q_full[s], (qi / C::NQ) & 1)) {
           ok = false;
           break;
