@@ -324,7 +324,9 @@ def capture_graph(call, device) -> torch.cuda.CUDAGraph:
     nothing; replaying the graph repeats the call's launches with the same arguments."""
     with torch.cuda.device(device):
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        # thread_local: CUDA calls other threads make meanwhile (a process group's watchdog, for one) are not
+        # checked against this capture
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
             call(None)
     return g
 
