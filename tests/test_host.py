@@ -165,6 +165,38 @@ def test_plan_with_splits_covers_every_row_once(case):
     _units_cover_exactly(*EDGE[case], split_ctas=1000)
 
 
+def _random_shapes(n, seed):
+    """Seeded random small layers: 1-3 sequences of up to 800 tokens (some with empty or whole-sequence query
+    ranges), G in {1, 2, 4, 8, 16}, D in {64, 128}, P in {16, 32, 64, 128}, and per (sequence, KV head) a global
+    head or a local one with a random sink (0 up to past the end) and window (1 up to past the end)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        B = int(rng.integers(1, 4))
+        seqs = []
+        for _ in range(B):
+            L = int(rng.integers(1, 801))
+            Lq = int(rng.choice([0, 1, L, int(rng.integers(0, L + 1))]))
+            seqs.append((L, Lq))
+        Hkv = int(rng.integers(1, 4))
+        G = int(rng.choice([1, 2, 4, 8, 16]))
+        D = int(rng.choice([64, 128]))
+        P = int(rng.choice([16, 32, 64, 128]))
+        classes = [[(1, 0, 0) if rng.random() < 0.3 else (0, int(rng.integers(0, 300)), int(rng.integers(1, 900)))
+                    for _ in range(Hkv)] for _ in range(B)]
+        split = int(rng.choice([0, 148, 1000]))
+        out.append((seqs, Hkv * G, Hkv, D, P, classes, split))
+    return out
+
+
+@pytest.mark.parametrize("case", range(24))
+def test_plan_covers_every_row_once_on_random_shapes(case):
+    """The planner's exact-cover and visible-key properties (as on the edge shapes) on seeded random layers,
+    with and without splitting."""
+    seqs, Hq, Hkv, D, P, classes, split = _random_shapes(24, 20251203)[case]
+    _units_cover_exactly(seqs, Hq, Hkv, D, P, classes, split_ctas=split)
+
+
 def test_split_policy_on_workloads():
     """Long-context prefill is never split; decode-like tiles and the 8K layer are."""
     def plan(w):
@@ -314,7 +346,16 @@ def test_mass_plan_covers_every_query_key_and_every_viewer(case):
     an item's query tiles [t0, t0 + nt) include every query tile with a row that sees one of those
     keys (the oracle's visibility rule) and start and end on such tiles; the key pages it reads are
     stored, at the table index the storage order gives; items come longest first."""
-    w_seqs, Hq, Hkv, D, P, classes = EDGE[case]
+    _mass_plan_check(*EDGE[case])
+
+
+@pytest.mark.parametrize("case", range(12))
+def test_mass_plan_on_random_shapes(case):
+    seqs, Hq, Hkv, D, P, classes, _ = _random_shapes(12, 20251204)[case]
+    _mass_plan_check(seqs, Hq, Hkv, D, P, classes)
+
+
+def _mass_plan_check(w_seqs, Hq, Hkv, D, P, classes):
     B = len(w_seqs)
     dims = sp.Dims(B, Hq, Hkv, D, P)
     ctx = [s[0] for s in w_seqs]
@@ -373,7 +414,16 @@ def test_append_plan_reads_old_keys_from_pool_and_new_keys_fresh(case, split):
     """Fused append-and-attend plan: a unit's page list holds only pages with a key before q0; its new pages
     (read from the new K/V) are consecutive logical pages from the first visible key at or after q0 to its
     last row; together they hold every visible key of every row (the oracle's sets); rows are covered once."""
-    w_seqs, Hq, Hkv, D, P, classes = EDGE[case]
+    _append_plan_check(*EDGE[case], split)
+
+
+@pytest.mark.parametrize("case", range(12))
+def test_append_plan_on_random_shapes(case):
+    seqs, Hq, Hkv, D, P, classes, split = _random_shapes(12, 20251205)[case]
+    _append_plan_check(seqs, Hq, Hkv, D, P, classes, split)
+
+
+def _append_plan_check(w_seqs, Hq, Hkv, D, P, classes, split):
     B = len(w_seqs)
     dims = sp.Dims(B, Hq, Hkv, D, P)
     ctx = [s[0] for s in w_seqs]
